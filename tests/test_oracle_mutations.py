@@ -1,0 +1,110 @@
+"""Plant plausible mistakes in a private copy of the oracle (on the CPU) and
+check that independent pins reject every one of them."""
+
+import importlib.util
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import softmax
+
+import oracle.attention as att
+import oracle.tokenizer as tok
+
+SRC_ATT = open(att.__file__).read()
+SRC_TOK = open(tok.__file__).read()
+
+
+def _load_mutant(src, name):
+    spec = importlib.util.spec_from_loader(name, loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    exec(compile(src, name, "exec"), mod.__dict__)
+    return mod
+
+
+def _fwd_pin_fails(mod):
+    """Softmax over the visible keys enumerated by hand, with a length mask."""
+    rng = np.random.default_rng(0)
+    n, d, R, L = 128, 8, 1, 90
+    q, k, v = (rng.standard_normal((1, 1, n, d)) for _ in range(3))
+    o, lse = mod.attn_fwd_dense(q, k, v, R, lengths=[L])
+    o_b, _ = mod.attn_fwd_banded(q, k, v, R, lengths=[L])
+    for i in range(L):
+        ib = i // 32
+        keys = [j for j in range(L) if abs(j // 32 - ib) <= R]
+        s = np.array([q[0, 0, i] @ k[0, 0, j] for j in keys]) / math.sqrt(d)
+        want = softmax(s) @ v[0, 0, keys]
+        if not (np.allclose(o[0, 0, i], want, atol=1e-10) and np.allclose(o_b[0, 0, i], want, atol=1e-10)):
+            return True
+    return False
+
+
+def _bwd_pin_fails(mod):
+    """Central differences of sum(O * dO) on a tiny case, for both oracles."""
+    rng = np.random.default_rng(1)
+    n, d, R, L = 64, 4, 0, 50
+    q, k, v, do = (rng.standard_normal((1, 1, n, d)) for _ in range(4))
+    h = 1e-6
+
+    def loss(qq, kk, vv):
+        o, _ = att.attn_fwd_dense(qq, kk, vv, R, lengths=[L])  # the unmutated forward
+        return float((o * do).sum())
+
+    for fn in (mod.attn_bwd_dense, mod.attn_bwd_banded):
+        grads = fn(q, k, v, do, R, lengths=[L])
+        for which, g in enumerate(grads):
+            for (i, t) in [(3, 1), (40, 2), (33, 0), (49, 3)]:
+                p = [q.copy(), k.copy(), v.copy()]
+                m = [q.copy(), k.copy(), v.copy()]
+                p[which][0, 0, i, t] += h
+                m[which][0, 0, i, t] -= h
+                fd = (loss(*p) - loss(*m)) / (2 * h)
+                if abs(fd - g[0, 0, i, t]) > 1e-6 * (1 + abs(fd)):
+                    return True
+    return False
+
+
+ATT_MUTATIONS = [
+    ("band off by one", "<= R\n    if length", "< R\n    if length"),
+    ("band j1 off by one", "min(nb - 1, i + R)", "min(nb - 1, i + R - 1)"),
+    ("scale dropped", "scale = 1.0 / math.sqrt(d)", "scale = 1.0"),
+    ("keys past length kept", "k0, k1 = j0 * BLOCK, min((j1 + 1) * BLOCK, L)  # keys past L are masked",
+     "k0, k1 = j0 * BLOCK, (j1 + 1) * BLOCK"),
+    ("length mask dropped", "m &= (np.arange(n) < length)[None, :]", "pass"),
+    ("D sign", "dS = P * (dP - D[:, None])  # softmax gradient", "dS = P * (dP + D[:, None])  # softmax gradient"),
+    ("D sign banded", "dS = P * (dP - D[:, None])\n", "dS = P * (dP + D[:, None])\n"),
+    ("D dropped", "dS = P * (dP - D[:, None])  # softmax gradient", "dS = P * dP  # softmax gradient"),
+    ("dK transposed", "dk[b, h] = scale * (dS.T @ q[b, h])", "dk[b, h] = scale * (dS @ q[b, h])"),
+    ("dV without P^T", "dv[b, h] = P.T @ dO", "dv[b, h] = P @ dO"),
+    ("dQ scale dropped", "dq[b, h] = scale * (dS @ k[b, h])", "dq[b, h] = dS @ k[b, h]"),
+    ("banded dK scale dropped", "dk[b, h, k0:k1] += scale * (dS.T @ Qi)", "dk[b, h, k0:k1] += dS.T @ Qi"),
+    ("softmax not normalised", "E / np.where(l > 0, l, 1.0)[:, None]", "E"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", ATT_MUTATIONS, ids=[m[0] for m in ATT_MUTATIONS])
+def test_attention_mutation_is_caught(name, old, new):
+    assert old in SRC_ATT, name
+    mod = _load_mutant(SRC_ATT.replace(old, new), "mutant_" + name.replace(" ", "_"))
+    assert _fwd_pin_fails(mod) or _bwd_pin_fails(mod), name
+
+
+TOK_MUTATIONS = [
+    ("code order", 'zip(b"ACGT", range(4))', 'zip(b"ACTG", range(4))'),
+    ("LSB first", "4 ** (k - 1 - t)", "4 ** t"),
+    ("flag value", "ids[bad] = N_FLAG_BASE ** k", "ids[bad] = 0"),
+    ("pack order", "(quads[:, 0] << 6) | (quads[:, 1] << 4) | (quads[:, 2] << 2) | quads[:, 3]",
+     "(quads[:, 3] << 6) | (quads[:, 2] << 4) | (quads[:, 1] << 2) | quads[:, 0]"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", TOK_MUTATIONS, ids=[m[0] for m in TOK_MUTATIONS])
+def test_tokenizer_mutation_is_caught(name, old, new):
+    assert old in SRC_TOK, name
+    mod = _load_mutant(SRC_TOK.replace(old, new), "mutant_tok")
+    page = {"TGGGAC": 3745, "TGAAGT": 3595, "GGCCCC": 2645}
+    ok = all(mod.kmer_ids(s.encode(), 6).tolist() == [v] for s, v in page.items())
+    ok &= mod.kmer_ids(b"ACGTNA", 6).tolist() == [4096]
+    ok &= mod.pack_2bit(b"ACGTG").tolist() == [0x1B, 0x80]
+    assert not ok, name

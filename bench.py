@@ -1,0 +1,490 @@
+"""Benchmark of the hot path: k-mer tokenization of a batch plus banded
+block-sparse local attention forward + backward, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of every step of the path over one batch: nb_tokenize_kmer
+on the batch's DNA (batch x (n + 5) bases), nb_attn_fwd and nb_attn_bwd.  Inputs
+are seeded synthetic tensors resident in HBM; several input sets rotate so that
+each step reads inputs that are not L2-resident.  Time is taken with CUDA
+events on the launching stream, bracketed by a barrier and a device
+synchronize, and the max over ranks is reported.  For N > 1 every rank
+processes its own batch (weak scaling, no collective on the data path).
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle (fp64
+NumPy) on a bounded sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse local attn fwd+bwd tokens/s and % of roofline (HBM or tensor)"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_local_nb_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/, valid
+    only while the kernel sources still hash to the value recorded with it."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    src = kernel_source_hash()
+    for line in lines:
+        parts = [p.strip() for p in line.strip().strip("|").split("|")]
+        if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[3] == src:
+            try:
+                return float(parts[2])
+            except ValueError:
+                return None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.device_index = device_index
+
+    def __enter__(self):
+        try:
+            import torch
+
+            props = torch.cuda.get_device_properties(self.device_index)
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            sel = ["--id=" + bus]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload
+
+def algorithmic(w, lengths):
+    """Algorithmic bytes and flops of one call (valid rows and visible pairs only)."""
+    e = 2 if w.dtype == "bf16" else 4
+    nb_ = w.n // 32
+    tok = 0
+    pairs = 0
+    for L in lengths:
+        L = int(L)
+        tok += L
+        for i in range((L + 31) // 32):
+            rows = min(32, L - 32 * i)
+            lo, hi = max(0, i - w.R), min(nb_ - 1, i + w.R)
+            keys = min((hi + 1) * 32, L) - lo * 32
+            pairs += rows * keys
+    th = tok * w.heads
+    pairs *= w.heads
+    return {
+        "tokens": tok,
+        "fwd_bytes": th * (4 * w.d * e + 4),   # read Q K V, write O and lse
+        "bwd_bytes": th * (8 * w.d * e + 4),   # read Q K V O dO lse, write dQ dK dV
+        "fwd_flops": 4 * w.d * pairs,          # Q K^T and P V
+        "bwd_flops": 10 * w.d * pairs,         # S, dP, dV, dK, dQ
+        "pairs": pairs,
+    }
+
+
+def dna_for_batch(w, seed):
+    from block_sparse_local_nb_b200.inputs import make_dna
+
+    return make_dna(w.batch * (w.n + 5), seed=seed)
+
+
+def run_reference_arm(args, w):
+    """Time the CPU oracle on a bounded sample of the workload (rank 0 only)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from block_sparse_local_nb_b200.inputs import make_attn_inputs
+    from oracle import attn_bwd_banded, attn_fwd_banded, kmer_ids, pack_2bit
+
+    q, k, v, do, lengths = make_attn_inputs(w)
+    dna = dna_for_batch(w, seed=w.seed)
+    lengths = lengths.numpy()
+    qn, kn, vn, don = (t.double().numpy() for t in (q, k, v, do))
+
+    def one(step):
+        # sample: one head of one sequence (rotating), plus that sequence's tokenization
+        b = step % w.batch
+        h = (step // w.batch) % w.heads
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        Lb = [int(lengths[b])]
+        attn_fwd_banded(qn[sl], kn[sl], vn[sl], w.R, Lb)
+        attn_bwd_banded(qn[sl], kn[sl], vn[sl], don[sl], w.R, Lb)
+        seg = dna[b * (w.n + 5):(b + 1) * (w.n + 5)]
+        kmer_ids(seg, 6)
+        pack_2bit(seg)
+        return Lb[0] / w.heads  # token-equivalents (a token = all heads of one position)
+
+    for s in range(args.warmup):
+        one(s)
+    t0 = time.perf_counter()
+    tok = 0.0
+    for s in range(args.steps):
+        tok += one(args.warmup + s)
+    dt = time.perf_counter() - t0
+    value = tok / dt
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "desc": w.desc, "batch": w.batch, "heads": w.heads,
+                   "n": w.n, "d": w.d, "R": w.R},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": "per step: one (sequence, head) of the batch through the fp64 "
+                                   "banded oracle forward+backward plus that sequence's k-mer "
+                                   "tokenization; counted as length/heads tokens"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w):
+    """Oracle timed on the host cores on a bounded sample (~10 s of CPU work)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from block_sparse_local_nb_b200.inputs import make_attn_inputs
+    from oracle import attn_bwd_banded, attn_fwd_banded, kmer_ids, pack_2bit
+
+    q, k, v, do, lengths = make_attn_inputs(w)
+    lengths = lengths.numpy()
+    dna = dna_for_batch(w, seed=w.seed)
+    qn, kn, vn, don = (t.double().numpy() for t in (q, k, v, do))
+    t0 = time.perf_counter()
+    tok = 0.0
+    heads_done = 0
+    budget = 10.0
+    while time.perf_counter() - t0 < budget and heads_done < w.batch * w.heads:
+        b, h = heads_done % w.batch, heads_done // w.batch
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        Lb = [int(lengths[b])]
+        attn_fwd_banded(qn[sl], kn[sl], vn[sl], w.R, Lb)
+        attn_bwd_banded(qn[sl], kn[sl], vn[sl], don[sl], w.R, Lb)
+        if h == 0:
+            seg = dna[b * (w.n + 5):(b + 1) * (w.n + 5)]
+            kmer_ids(seg, 6)
+            pack_2bit(seg)
+        tok += Lb[0] / w.heads
+        heads_done += 1
+    dt = time.perf_counter() - t0
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    return {"value": tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{heads_done} of {w.batch * w.heads} (sequence, head) pairs through the fp64 "
+                      f"banded oracle fwd+bwd plus per-sequence k-mer tokenization, {dt:.1f} s; "
+                      f"host has {os.cpu_count()} logical cores"}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="bf16_varlen")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--sets", type=int, default=0, help="rotating input sets (0 = auto)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    from block_sparse_local_nb_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference_arm(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_local_nb_b200 as nb
+    from block_sparse_local_nb_b200.inputs import make_attn_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    dt_code = nb.NB_BF16 if w.dtype == "bf16" else nb.NB_F32
+    B, H, N, D, R = w.batch, w.heads, w.n, w.d, w.R
+    stream = torch.cuda.Stream(device=dev)
+
+    # ---- resident inputs: rotating sets so each step's reads miss L2
+    per_set = None
+    sets = []
+    base_seed = w.seed + 1000 * rank
+    nsets = args.sets
+    q0, k0, v0, do0, lengths = make_attn_inputs(w, device=dev, seed=base_seed)
+    lengths_d = lengths.to(dev)
+    dna_np = dna_for_batch(w, seed=base_seed)
+    elem = q0.element_size()
+    set_bytes = (8 * q0.numel() * elem + 2 * B * H * N * 4
+                 + nb.attn_bwd_workspace_size(B, H, N, D, dt_code) + 3 * dna_np.size)
+    if nsets <= 0:
+        nsets = max(1, min(8, math.ceil(3 * L2_BYTES / set_bytes) + 1))
+    for s in range(nsets):
+        if s == 0:
+            q, k, v, do = q0, k0, v0, do0
+        else:
+            q, k, v, do, _ = make_attn_inputs(w, device=dev, seed=base_seed + s)
+        st = {"q": q, "k": k, "v": v, "do": do,
+              "o": torch.empty_like(q), "lse": torch.empty((B, H, N), dtype=torch.float32, device=dev),
+              "dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+              "dna": torch.from_numpy(dna_np).to(dev),
+              "ids": torch.empty(dna_np.size - 5, dtype=torch.int16, device=dev),
+              "packed": torch.empty((dna_np.size + 3) // 4, dtype=torch.uint8, device=dev)}
+        ws_bytes = nb.attn_bwd_workspace_size(B, H, N, D, dt_code)
+        st["ws"] = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+        st["ws_bytes"] = ws_bytes
+        sets.append(st)
+    torch.cuda.synchronize(dev)
+
+    sptr = stream.cuda_stream
+
+    def step(st, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        nb.nb_tokenize_kmer(st["dna"], st["dna"].numel(), st["ids"], st["packed"], 6, sptr)
+        if ev is not None:
+            ev[1].record(stream)
+        nb.nb_attn_fwd(st["q"], st["k"], st["v"], st["o"], st["lse"], lengths_d, B, H, N, D, R,
+                       dt_code, sptr)
+        if ev is not None:
+            ev[2].record(stream)
+        if w.backward:
+            nb.nb_attn_bwd(st["q"], st["k"], st["v"], st["o"], st["do"], st["lse"], lengths_d,
+                           st["dq"], st["dk"], st["dv"], st["ws"], st["ws_bytes"], B, H, N, D, R,
+                           dt_code, sptr)
+        if ev is not None:
+            ev[3].record(stream)
+
+    launches_per_step = 1 + 1 + (3 if w.backward else 0)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize(dev)
+
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            step(sets[s % nsets])
+    barrier()
+
+    # ---- timed region: exactly K steps, per-call events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        barrier()
+        start.record(stream)
+        for s in range(args.steps):
+            step(sets[s % nsets], evs[s])
+        end.record(stream)
+        barrier()
+    elapsed_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    tok_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+
+    alg = algorithmic(w, lengths.tolist())
+    tokens_step = alg["tokens"]
+    value = tokens_step * args.steps * world / (elapsed_ms / 1e3)
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies timed
+    host = {}
+    for name in ("q", "k", "v", "do"):
+        host[name] = sets[0][name].cpu().pin_memory()
+    host["dna"] = torch.from_numpy(dna_np).pin_memory()
+    host["lengths"] = lengths.pin_memory()
+    outs = {name: torch.empty_like(sets[0][name], device="cpu").pin_memory()
+            for name in ("o", "lse", "dq", "dk", "dv", "ids", "packed")}
+    st = sets[0]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            for name in ("q", "k", "v", "do", "dna"):
+                st[name].copy_(host[name], non_blocking=True)
+            lengths_d.copy_(host["lengths"], non_blocking=True)
+            step(st)
+            for name, t in outs.items():
+                t.copy_(st[name], non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        e_start.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e_end.record(stream)
+        barrier()
+    e2e_ms = e_start.elapsed_time(e_end)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = tokens_step * args.steps * world / (e2e_ms / 1e3)
+
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    bf16 = float(peaks["bf16_tflops"])
+    fwd_avg = statistics.mean(fwd_ms)
+    bwd_avg = statistics.mean(bwd_ms) if w.backward else 0.0
+    tok_avg = statistics.mean(tok_ms)
+    # dominant call of the step
+    if w.backward and bwd_avg >= fwd_avg:
+        dom, dom_ms, dom_bytes, dom_flops = "nb_attn_bwd", bwd_avg, alg["bwd_bytes"], alg["bwd_flops"]
+    else:
+        dom, dom_ms, dom_bytes, dom_flops = "nb_attn_fwd", fwd_avg, alg["fwd_bytes"], alg["fwd_flops"]
+    t_hbm = dom_bytes / (hbm * 1e9)
+    t_tc = dom_flops / (bf16 * 1e12)
+    if t_hbm >= t_tc:
+        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s"}
+    else:
+        achieved = dom_flops / (dom_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic(dom, w.name)
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'fallback'})"
+
+    step_bytes = alg["fwd_bytes"] + (alg["bwd_bytes"] if w.backward else 0)
+    step_flops = alg["fwd_flops"] + (alg["bwd_flops"] if w.backward else 0)
+    ms_per_step = elapsed_ms / args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "desc": w.desc + " + k=6 tokenization of the batch's "
+                   f"{B}x({N}+5) bases", "batch": B, "heads": H, "n": N, "d": D, "R": R,
+                   "tokens_per_step": tokens_step, "parallelism": f"dp{world} (independent batches)",
+                   "l2": f"{nsets} rotating input sets of {set_bytes / 2**20:.0f} MiB each "
+                         f"(> {L2_BYTES >> 20} MiB L2 between reuses)"},
+        "roofline": roof,
+        "step_roofline": {"bytes": step_bytes, "flops": step_flops,
+                          "hbm_frac": step_bytes / (ms_per_step / 1e3) / (hbm * 1e9),
+                          "tensor_frac": step_flops / (ms_per_step / 1e3) / (bf16 * 1e12),
+                          "frac_of_roofline": max(step_bytes / (hbm * 1e9), step_flops / (bf16 * 1e12))
+                          / (ms_per_step / 1e3)},
+        "calls_ms": {"nb_tokenize_kmer": tok_avg, "nb_attn_fwd": fwd_avg, "nb_attn_bwd": bwd_avg},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,147 @@
+// C ABI of the library (declared in include/nb.h): host-side argument
+// validation, device check and dispatch to the kernel launchers.  Everything
+// here runs on the host before any launch, so an invalid call launches nothing.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/nb.h"
+#include "nb_internal.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+// Per-device cache: 0 = unknown, 1 = sm_100 (supported), -1 = other.
+int g_device_ok[kMaxDevices];
+
+nb_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NB_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return NB_ERR_DEVICE;
+  int state = __atomic_load_n(&g_device_ok[dev], __ATOMIC_RELAXED);
+  if (state == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return NB_ERR_CUDA;
+    state = (major == 10 && minor == 0) ? 1 : -1;
+    __atomic_store_n(&g_device_ok[dev], state, __ATOMIC_RELAXED);
+  }
+  return state == 1 ? NB_OK : NB_ERR_DEVICE;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by forward and backward.
+nb_status check_shape(int batch, int heads, int n, int d, int R, int dtype) {
+  if (batch < 0 || heads < 0 || n < 0 || R < 0) return NB_ERR_INVALID_ARG;
+  if (n % nb::kBlock != 0) return NB_ERR_INVALID_ARG;
+  if (dtype != NB_F32 && dtype != NB_BF16) return NB_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return NB_ERR_UNSUPPORTED;
+  if (heads > 65535 || batch > 65535) return NB_ERR_UNSUPPORTED;  // grid y / z limits
+  // element count must fit comfortably in int64 and rows*d*4 in size_t
+  const double elems = static_cast<double>(batch) * heads * n * d;
+  if (elems > 9.0e15) return NB_ERR_INVALID_ARG;
+  return NB_OK;
+}
+
+nb::AttnArgs make_args(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, const int32_t* lengths, void* dq,
+                       void* dk, void* dv, void* ws, int batch, int heads, int n, int d, int R) {
+  nb::AttnArgs a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout;
+  a.lse = const_cast<float*>(lse);
+  a.lengths = lengths;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.workspace = ws;
+  a.batch = batch; a.heads = heads; a.n = n; a.d = d; a.R = R;
+  a.scale = static_cast<float>(1.0 / sqrt(static_cast<double>(d)));
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nb_status_string(int status) {
+  switch (status) {
+    case NB_OK: return "NB_OK";
+    case NB_ERR_INVALID_ARG: return "NB_ERR_INVALID_ARG: invalid argument";
+    case NB_ERR_UNSUPPORTED: return "NB_ERR_UNSUPPORTED: unsupported configuration";
+    case NB_ERR_MISALIGNED: return "NB_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case NB_ERR_CUDA: return "NB_ERR_CUDA: CUDA runtime error";
+    case NB_ERR_WORKSPACE: return "NB_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case NB_ERR_DEVICE: return "NB_ERR_DEVICE: current device is not sm_100";
+    default: return "unknown nb_status";
+  }
+}
+
+int nb_abi_version(void) { return 100; }
+
+nb_status nb_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                      const int32_t* lengths, int batch, int heads, int n, int d, int R,
+                      int dtype, void* stream) {
+  nb_status st = check_shape(batch, heads, n, d, R, dtype);
+  if (st != NB_OK) return st;
+  if (static_cast<int64_t>(batch) * heads * n == 0) return NB_OK;
+  if (!q || !k || !v || !o) return NB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && !aligned16(lse)) || (lengths && (reinterpret_cast<uintptr_t>(lengths) & 3u)))
+    return NB_ERR_MISALIGNED;
+  st = check_device();
+  if (st != NB_OK) return st;
+  nb::AttnArgs a = make_args(q, k, v, o, nullptr, lse, lengths, nullptr, nullptr, nullptr,
+                             nullptr, batch, heads, n, d, R);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = dtype == NB_F32 ? nb::launch_attn_fwd_f32(a, s) : nb::launch_attn_fwd_bf16(a, s);
+  return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
+}
+
+size_t nb_attn_bwd_workspace_size(int batch, int heads, int n, int d, int dtype) {
+  if (check_shape(batch, heads, n, d, 0, dtype) != NB_OK) return 0;
+  const int64_t rows = static_cast<int64_t>(batch) * heads * n;
+  if (rows == 0) return 0;
+  return nb::bwd_workspace_bytes(rows, d);
+}
+
+nb_status nb_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, const int32_t* lengths, void* dq,
+                      void* dk, void* dv, void* workspace, size_t workspace_bytes, int batch,
+                      int heads, int n, int d, int R, int dtype, void* stream) {
+  nb_status st = check_shape(batch, heads, n, d, R, dtype);
+  if (st != NB_OK) return st;
+  if (static_cast<int64_t>(batch) * heads * n == 0) return NB_OK;
+  if (dtype != NB_BF16) return NB_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return NB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (lengths && (reinterpret_cast<uintptr_t>(lengths) & 3u)))
+    return NB_ERR_MISALIGNED;
+  const int64_t rows = static_cast<int64_t>(batch) * heads * n;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < nb::bwd_workspace_bytes(rows, d))
+    return NB_ERR_WORKSPACE;
+  st = check_device();
+  if (st != NB_OK) return st;
+  nb::AttnArgs a = make_args(q, k, v, o, dout, lse, lengths, dq, dk, dv, workspace, batch, heads,
+                             n, d, R);
+  cudaError_t e = nb::launch_attn_bwd_bf16(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
+}
+
+nb_status nb_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
+                           int k, void* stream) {
+  if (len < 0) return NB_ERR_INVALID_ARG;
+  if (k < 1 || k > 7) return NB_ERR_UNSUPPORTED;
+  if (ids && (reinterpret_cast<uintptr_t>(ids) & 1u)) return NB_ERR_MISALIGNED;
+  if (len == 0 || (!ids && !packed)) return NB_OK;
+  if (!seq) return NB_ERR_INVALID_ARG;
+  if (len < k) ids = nullptr;  // no complete window: only the packed stream is written
+  if (!ids && !packed) return NB_OK;
+  nb_status st = check_device();
+  if (st != NB_OK) return st;
+  cudaError_t e =
+      nb::launch_tokenize_kmer(seq, len, ids, packed, k, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,145 @@
+/*
+ * nb.h - C ABI of the B200 (sm_100a) banded block-sparse local attention and
+ * the fused 2-bit DNA k-mer tokenizer.
+ *
+ * The operations follow the NucleoByte page ("NucleoByte: GPU-Accelerated
+ * Block-Sparse Genomic Language Model"):
+ *   - section 3 "Mathematical Foundations", subsection "Localized Block-Sparse
+ *     Attention Matrix": blocks of B = 32 tokens; query block i attends key
+ *     block j only when |i - j| <= R;
+ *   - section 3, "Softmax Normalization & Online Numerical Stability":
+ *     S = Q K^T / sqrt(d), online softmax with running max and running sum;
+ *   - section 3, "Custom Backpropagation": row term D_i = sum_k dO_ik O_ik and
+ *     dS_ij = P_ij (dO_i V_j^T - D_i);
+ *   - sections 1-2 ("Padding Waste", "Dynamic Ceiling Hardware Alignment"):
+ *     sequences padded to a multiple of 32, keys past the true length masked;
+ *   - sections 1, 2 and 5 ("Token Blur", "Fused 2-Bit Tokenization",
+ *     "Architecture Size"): 2-bit bases, sliding-window 6-mer IDs.
+ *
+ * Conventions shared by every call:
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise.  The
+ *     caller owns every buffer; the library keeps no state between calls except
+ *     a per-device cache of device properties, and allocates no device memory.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Arguments are validated on the host first: an invalid
+ *     call returns a negative nb_status and launches nothing.  A failed launch
+ *     returns NB_ERR_CUDA.  Kernels never trap.
+ *   - Attention tensors are [batch, heads, n, d] contiguous with d innermost;
+ *     log-sum-exp and the row term are [batch, heads, n] fp32.  n must be a
+ *     multiple of 32 and d is 64 or 128.  Tensor pointers must be 16-byte
+ *     aligned.
+ *   - `lengths` (optional, int32 [batch], device) gives each sequence's true
+ *     length L_b in [0, n]; NULL means every L_b = n.  Keys k >= L_b are
+ *     masked.  Rows q >= L_b are padding: O, dQ, dK, dV are written as 0 there
+ *     and log-sum-exp as -inf.  Values outside [0, n] are clamped into it on
+ *     the device (they cannot be checked on the host).
+ *   - The softmax scale is fixed at 1/sqrt(d).
+ */
+#ifndef NB_H_
+#define NB_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NB_API __attribute__((visibility("default")))
+#else
+#define NB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum nb_status {
+  NB_OK = 0,
+  NB_ERR_INVALID_ARG = -1, /* null pointer, bad size, n % 32 != 0, R < 0, ... */
+  NB_ERR_UNSUPPORTED = -2, /* valid request this build does not implement (d, dtype, k) */
+  NB_ERR_MISALIGNED = -3,  /* a tensor pointer is not 16-byte aligned */
+  NB_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+  NB_ERR_WORKSPACE = -5,   /* workspace pointer null/misaligned or too small */
+  NB_ERR_DEVICE = -6       /* the current device is not an sm_100 (B200-class) GPU */
+} nb_status;
+
+typedef enum nb_dtype {
+  NB_F32 = 0,  /* fp32 storage, fp32 arithmetic (CUDA cores) */
+  NB_BF16 = 1  /* bf16 storage, fp32 accumulation (tensor cores) */
+} nb_dtype;
+
+#define NB_BLOCK 32 /* the block size B of the band */
+
+/* Human-readable name of a status code.  Never returns NULL. */
+NB_API const char* nb_status_string(int status);
+
+/* ABI version of this library (major * 100 + minor). */
+NB_API int nb_abi_version(void);
+
+/*
+ * nb_attn_fwd - banded block-sparse local attention, forward.
+ *   O[b,h,q,:] = sum_k P[q,k] V[b,h,k,:], P = softmax over the visible keys of
+ *   S = Q K^T / sqrt(d); visible: |q/32 - k/32| <= R and k < L_b.
+ *   (NucleoByte page, section 3: band predicate, scores, online softmax.)
+ * q, k, v  in : [batch, heads, n, d] of `dtype`.
+ * o        out: [batch, heads, n, d] of `dtype`.
+ * lse      out: [batch, heads, n] fp32, natural-log log-sum-exp of each row's
+ *               visible scaled scores (the input the backward needs); may be
+ *               NULL when not wanted.
+ * lengths  in : int32 [batch] or NULL (see conventions).
+ * batch, heads >= 0; n >= 0 and a multiple of 32; d in {64, 128}; R >= 0.
+ * dtype: NB_F32 or NB_BF16.  stream: cudaStream_t.
+ * Empty problems (batch*heads*n == 0) return NB_OK without a launch.
+ */
+NB_API nb_status nb_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                      const int32_t* lengths, int batch, int heads, int n, int d, int R,
+                      int dtype, void* stream);
+
+/*
+ * nb_attn_bwd_workspace_size - bytes of device workspace nb_attn_bwd needs
+ * for this shape (0 for an empty problem).  Returns 0 for invalid arguments.
+ */
+NB_API size_t nb_attn_bwd_workspace_size(int batch, int heads, int n, int d, int dtype);
+
+/*
+ * nb_attn_bwd - backward of nb_attn_fwd, recomputing P from the stored
+ * log-sum-exp.  (NucleoByte page, section 3 "Custom Backpropagation":
+ * D_i = sum_k dO_ik O_ik, dS = P (dO V^T - D); dV = P^T dO, dQ = dS K / sqrt(d),
+ * dK = dS^T Q / sqrt(d).)
+ * q, k, v   in : the forward's inputs.
+ * o, lse    in : the forward's outputs for the same inputs (lse required).
+ * dout      in : dL/dO, [batch, heads, n, d] of `dtype`; rows >= L_b ignored.
+ * dq, dk, dv out: [batch, heads, n, d] of `dtype`; must not alias the inputs.
+ * workspace     : device scratch of at least nb_attn_bwd_workspace_size(...)
+ *                 bytes, 256-byte aligned, owned by the caller; its contents on
+ *                 entry do not matter and are clobbered.  It must not be used
+ *                 by another call that runs concurrently on the GPU.
+ * dK and dV are deterministic; dQ is accumulated with fp32 atomics and may
+ * differ in the last bits between runs.
+ * Currently NB_BF16 only (NB_F32 returns NB_ERR_UNSUPPORTED).
+ */
+NB_API nb_status nb_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, const int32_t* lengths, void* dq,
+                      void* dk, void* dv, void* workspace, size_t workspace_bytes, int batch,
+                      int heads, int n, int d, int R, int dtype, void* stream);
+
+/*
+ * nb_tokenize_kmer - fused 2-bit DNA k-mer tokenizer.
+ * (NucleoByte page, sections 1 "Token Blur", 2 "Fused 2-Bit Tokenization",
+ * 5 "Architecture Size" and "Evaluation Output Verification".)
+ * seq     in : len ASCII bytes (any alignment).  A=0, C=1, G=2, T=3; any other
+ *              byte is invalid.
+ * ids     out: uint16 [len - k + 1] (nothing when len < k) or NULL: window p has
+ *              ID sum_t code[p+t] * 4^(k-1-t) (first base most significant), or
+ *              4^k when the window holds an invalid byte.
+ * packed  out: uint8 [(len + 3) / 4] or NULL: 4 bases per byte, first base in
+ *              bits 7..6, invalid bases stored as 0, unused tail slots 0.
+ * k: 1..7 (the page uses 6).  len >= 0.  ids must be 2-byte aligned.
+ * Both outputs NULL is valid and does nothing.
+ */
+NB_API nb_status nb_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
+                           int k, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NB_H_ */

@@ -1,0 +1,136 @@
+"""CPU checks of the C-ABI library: it loads, exports every function that
+include/nb.h declares, and rejects invalid arguments on the host (these calls
+return before any CUDA call, so they run without a GPU)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "nb.h")
+LIB = os.path.join(ROOT, "block_sparse_local_nb_b200", "libnb_b200.so")
+
+NB_OK, NB_ERR_INVALID_ARG, NB_ERR_UNSUPPORTED, NB_ERR_MISALIGNED = 0, -1, -2, -3
+NB_ERR_WORKSPACE = -5
+F32, BF16 = 0, 1
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"NB_API\s+[\w\s\*]+?\b(nb_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from block_sparse_local_nb_b200.build import build
+
+        build()
+    from block_sparse_local_nb_b200 import binding
+
+    return binding.lib()
+
+
+def test_header_declares_the_abi():
+    names = _declared_functions()
+    assert {"nb_attn_fwd", "nb_attn_bwd", "nb_attn_bwd_workspace_size", "nb_tokenize_kmer",
+            "nb_status_string", "nb_abi_version"} <= set(names)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\sT\s(nb_\w+)", out))
+    for name in _declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_library_links_no_cuda_runtime_dynamically():
+    out = subprocess.run(["ldd", LIB], capture_output=True, text=True).stdout
+    assert "libcudart" not in out and "libtorch" not in out
+
+
+def test_status_strings(lib):
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.nb_status_string(st)
+    assert lib.nb_abi_version() >= 100
+
+
+def _fwd(lib, q=16, k=16, v=16, o=16, lse=None, lengths=None, batch=1, heads=1, n=64, d=64,
+         R=1, dtype=BF16):
+    return lib.nb_attn_fwd(q, k, v, o, lse, lengths, batch, heads, n, d, R, dtype, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n=48), NB_ERR_INVALID_ARG),        # n not a multiple of 32
+    (dict(n=-32), NB_ERR_INVALID_ARG),
+    (dict(R=-1), NB_ERR_INVALID_ARG),
+    (dict(batch=-1), NB_ERR_INVALID_ARG),
+    (dict(dtype=7), NB_ERR_INVALID_ARG),
+    (dict(d=32), NB_ERR_UNSUPPORTED),
+    (dict(d=96), NB_ERR_UNSUPPORTED),
+    (dict(q=None), NB_ERR_INVALID_ARG),
+    (dict(o=None), NB_ERR_INVALID_ARG),
+    (dict(k=24), NB_ERR_MISALIGNED),
+    (dict(lse=20), NB_ERR_MISALIGNED),
+    (dict(lengths=18), NB_ERR_MISALIGNED),
+    (dict(heads=70000), NB_ERR_UNSUPPORTED),
+])
+def test_fwd_rejects_invalid_arguments(lib, kw, status):
+    assert _fwd(lib, **kw) == status
+
+
+def test_fwd_empty_problem_is_a_no_op(lib):
+    assert _fwd(lib, batch=0) == NB_OK
+    assert _fwd(lib, heads=0, q=None, k=None, v=None, o=None) == NB_OK
+    assert _fwd(lib, n=0) == NB_OK
+
+
+def test_bwd_workspace_size(lib):
+    ws = lib.nb_attn_bwd_workspace_size(4, 12, 4096, 64, BF16)
+    rows = 4 * 12 * 4096
+    assert ws >= rows * 4 + rows * 64 * 4
+    assert ws < rows * 4 + rows * 64 * 4 + 1024
+    assert lib.nb_attn_bwd_workspace_size(1, 1, 33, 64, BF16) == 0  # invalid n
+    assert lib.nb_attn_bwd_workspace_size(0, 1, 64, 64, BF16) == 0
+
+
+def _bwd(lib, ws=256, ws_bytes=1 << 30, dq=16, lse=16, dtype=BF16, n=64, d=64, R=1, k=16):
+    return lib.nb_attn_bwd(16, k, 16, 16, 16, lse, None, dq, 16, 16, ws, ws_bytes, 1, 1, n, d, R,
+                           dtype, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ws=None), NB_ERR_WORKSPACE),
+    (dict(ws=272), NB_ERR_WORKSPACE),       # not 256-byte aligned
+    (dict(ws_bytes=100), NB_ERR_WORKSPACE),  # too small
+    (dict(lse=None), NB_ERR_INVALID_ARG),
+    (dict(dq=None), NB_ERR_INVALID_ARG),
+    (dict(dq=8), NB_ERR_MISALIGNED),
+    (dict(k=40), NB_ERR_MISALIGNED),
+    (dict(dtype=F32), NB_ERR_UNSUPPORTED),
+    (dict(n=40), NB_ERR_INVALID_ARG),
+    (dict(R=-2), NB_ERR_INVALID_ARG),
+])
+def test_bwd_rejects_invalid_arguments(lib, kw, status):
+    assert _bwd(lib, **kw) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    ((16, -1, 32, None, 6), NB_ERR_INVALID_ARG),
+    ((16, 100, 32, None, 0), NB_ERR_UNSUPPORTED),
+    ((16, 100, 32, None, 8), NB_ERR_UNSUPPORTED),
+    ((16, 100, 33, None, 6), NB_ERR_MISALIGNED),
+    ((None, 100, 32, None, 6), NB_ERR_INVALID_ARG),
+    ((16, 0, 32, 32, 6), NB_OK),
+    ((16, 100, None, None, 6), NB_OK),
+    ((16, 5, 32, None, 6), NB_OK),  # len < k with only ids: nothing to write
+])
+def test_tokenize_rejects_invalid_arguments(lib, args, status):
+    seq, n, ids, packed, k = args
+    assert lib.nb_tokenize_kmer(seq, n, ids, packed, k, None) == status

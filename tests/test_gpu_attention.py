@@ -1,0 +1,220 @@
+"""GPU parity of nb_attn_fwd / nb_attn_bwd against the fp64 oracle.
+
+Small cases compare every element; the full-size workloads compare sampled
+windows of blocks (the oracle evaluated on a sub-sequence with two band radii
+of context on each side, where its outputs are exact).  Tolerances:
+fp32 max-abs 1e-4 (O, lse); bf16 max-abs 1.5e-2 on O, 1e-3 on lse,
+relative Frobenius 1e-2 on dQ, dK, dV.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_local_nb_b200.inputs import WORKLOADS, make_attn_inputs, random_attn_inputs
+from oracle import attn_bwd_banded, attn_fwd_banded, attn_fwd_dense
+from tests.gpu_util import (ATOL_F32, GRAD_RFRO_BF16, LSE_ATOL_BF16, O_ATOL_BF16, f64, max_abs,
+                            rel_fro, run_bwd, run_fwd, window)
+
+pytestmark = pytest.mark.gpu
+BLOCK = 32
+
+
+def _lengths(vals):
+    return torch.tensor(vals, dtype=torch.int32)
+
+
+def _cuda(*ts):
+    return [t.cuda() for t in ts]
+
+
+# ------------------------------------------------------------------ fp32
+
+def test_fp32_n256_workload():
+    """fp32, 1 x 1 x 256 x 64, R = 1, full length, seed 0: every element."""
+    w = WORKLOADS["fp32_n256"]
+    q, k, v, _, lengths = make_attn_inputs(w)
+    o, lse = run_fwd(*_cuda(q, k, v), lengths, w.R)
+    o_ref, lse_ref = attn_fwd_dense(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                    w.R, lengths.numpy())
+    assert max_abs(f64(o), o_ref) <= ATOL_F32
+    assert max_abs(f64(lse), lse_ref) <= ATOL_F32
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n,R,lens", [
+    (32, 0, [32, 1]), (64, 1, [64, 33]), (96, 2, [0, 95]), (288, 2, [288, 200]),
+    (288, 9, [17, 288]), (160, 0, [160, 31]),
+])
+def test_fp32_small(n, R, lens, d):
+    q, k, v, _ = random_attn_inputs(2, 3, n, d, "f32", seed=n + R + d)
+    L = _lengths(lens)
+    o, lse = run_fwd(*_cuda(q, k, v), L, R)
+    o_ref, lse_ref = attn_fwd_dense(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                    R, L.numpy())
+    assert max_abs(f64(o), o_ref) <= ATOL_F32
+    assert max_abs(f64(lse), lse_ref) <= ATOL_F32
+
+
+# ----------------------------------------------------------------- bf16 small
+
+SMALL = [
+    (32, 0, [32]), (64, 1, [64, 1]), (96, 2, [96, 50]), (128, 1, [100, 128]),
+    (160, 1, [160, 0]), (288, 2, [288, 257]), (288, 9, [200, 288]), (416, 3, [33, 416]),
+    (512, 4, [512, 480]), (544, 8, [544, 321]),
+]
+
+
+def _bf16_case(n, R, lens, d, seed, heads=3):
+    q, k, v, do = random_attn_inputs(len(lens), heads, n, d, "bf16", seed=seed)
+    L = _lengths(lens)
+    qd, kd, vd, dod = _cuda(q, k, v, do)
+    o, lse = run_fwd(qd, kd, vd, L, R)
+    dq, dk, dv = run_bwd(qd, kd, vd, o, dod, lse, L, R)
+    args = [t.double().numpy() for t in (q, k, v)]
+    o_ref, lse_ref = attn_fwd_banded(*args, R, L.numpy())
+    grads_ref = attn_bwd_banded(*args, do.double().numpy(), R, L.numpy())
+    return (o, lse, dq, dk, dv), (o_ref, lse_ref, *grads_ref), L
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n,R,lens", SMALL)
+def test_bf16_fwd_bwd_small(n, R, lens, d):
+    got, ref, L = _bf16_case(n, R, lens, d, seed=7 * n + R + d)
+    o, lse, dq, dk, dv = got
+    o_ref, lse_ref, dq_ref, dk_ref, dv_ref = ref
+    assert max_abs(f64(o), o_ref) <= O_ATOL_BF16
+    assert max_abs(f64(lse), lse_ref) <= LSE_ATOL_BF16
+    for name, g, r in (("dq", dq, dq_ref), ("dk", dk, dk_ref), ("dv", dv, dv_ref)):
+        assert rel_fro(f64(g), r) <= GRAD_RFRO_BF16, name
+    # padding rows are exactly zero, log-sum-exp -inf
+    for b, Lb in enumerate(L.tolist()):
+        for t in (o, dq, dk, dv):
+            assert (t[b, :, Lb:] == 0).all()
+        assert torch.isneginf(lse[b, :, Lb:]).all()
+
+
+def test_bf16_dk_dv_deterministic():
+    q, k, v, do = _cuda(*random_attn_inputs(2, 4, 1024, 64, "bf16", seed=5))
+    L = _lengths([1024, 700])
+    o, lse = run_fwd(q, k, v, L, 2)
+    a = run_bwd(q, k, v, o, do, lse, L, 2)
+    b = run_bwd(q, k, v, o, do, lse, L, 2)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert rel_fro(f64(a[0]), f64(b[0])) < 1e-3
+    o2, lse2 = run_fwd(q, k, v, L, 2)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+
+
+def test_bf16_padding_contents_are_ignored():
+    """Garbage (1e4) in Q, K, V and dO past each length changes nothing."""
+    n, R, d = 640, 2, 64
+    q, k, v, do = _cuda(*random_attn_inputs(2, 2, n, d, "bf16", seed=9))
+    L = _lengths([500, 333])
+    o, lse = run_fwd(q, k, v, L, R)
+    grads = run_bwd(q, k, v, o, do, lse, L, R)
+    q2, k2, v2, do2 = (t.clone() for t in (q, k, v, do))
+    for b, Lb in enumerate(L.tolist()):
+        for t in (q2, k2, v2, do2):
+            t[b, :, Lb:] = 1e4
+    o2, lse2 = run_fwd(q2, k2, v2, L, R)
+    grads2 = run_bwd(q2, k2, v2, o2, do2, lse2, L, R)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+    assert torch.equal(grads[1], grads2[1]) and torch.equal(grads[2], grads2[2])
+    assert rel_fro(f64(grads2[0]), f64(grads[0])) < 1e-3
+
+
+def test_bf16_lse_optional_and_lengths_null():
+    n, R, d = 256, 1, 64
+    q, k, v, _ = _cuda(*random_attn_inputs(1, 2, n, d, "bf16", seed=4))
+    o_full, _ = run_fwd(q, k, v, None, R)
+    o_none, _ = run_fwd(q, k, v, _lengths([n]), R, with_lse=False)
+    assert torch.equal(o_full, o_none)
+
+
+def test_bf16_out_of_range_lengths_are_clamped():
+    n, R, d = 128, 1, 64
+    q, k, v, do = _cuda(*random_attn_inputs(2, 1, n, d, "bf16", seed=6))
+    o_a, lse_a = run_fwd(q, k, v, _lengths([n + 1000, -5]), R)
+    o_b, lse_b = run_fwd(q, k, v, _lengths([n, 0]), R)
+    assert torch.equal(o_a, o_b) and torch.equal(lse_a, lse_b)
+
+
+# ------------------------------------------------------- full-size workloads
+
+def _check_window(w, tensors, outs, bh, blk_lo, blk_hi, lengths, check_bwd=True):
+    """Compare the GPU outputs of one (batch, head) on blocks [blk_lo, blk_hi)."""
+    q, k, v, do = tensors
+    o, lse, dq, dk, dv = outs
+    b, h = bh
+    nb = w.n // BLOCK
+    s, e = window(nb, blk_lo, blk_hi, w.R)
+    Lb = int(lengths[b])
+    Lsub = min(max(Lb - s * BLOCK, 0), (e - s) * BLOCK)
+    sl = slice(s * BLOCK, e * BLOCK)
+    sub = [t[b, h, sl].double().cpu().numpy()[None, None] for t in (q, k, v, do)]
+    o_ref, lse_ref = attn_fwd_banded(*sub[:3], w.R, [Lsub])
+    r0, r1 = (blk_lo - s) * BLOCK, (blk_hi - s) * BLOCK
+    g0, g1 = blk_lo * BLOCK, blk_hi * BLOCK
+    assert max_abs(f64(o[b, h, g0:g1]), o_ref[0, 0, r0:r1]) <= O_ATOL_BF16
+    assert max_abs(f64(lse[b, h, g0:g1]), lse_ref[0, 0, r0:r1]) <= LSE_ATOL_BF16
+    if check_bwd:
+        grads_ref = attn_bwd_banded(*sub, w.R, [Lsub])
+        for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), grads_ref):
+            err = rel_fro(f64(g[b, h, g0:g1]), r[0, 0, r0:r1])
+            assert err <= GRAD_RFRO_BF16, (name, err)
+
+
+def _run_workload(w):
+    q, k, v, do, lengths = make_attn_inputs(w, device="cuda")
+    o, lse = run_fwd(q, k, v, lengths, w.R)
+    grads = run_bwd(q, k, v, o, do, lse, lengths, w.R) if w.backward else (None,) * 3
+    torch.cuda.synchronize()
+    return (q, k, v, do), (o, lse, *grads), lengths
+
+
+def test_bf16_varlen_workload():
+    """bf16, 4 x 12 x 4096 x 64, R = 2, lengths ~ U[1024, 4096]: three whole heads
+    and sampled windows of the rest, including each sequence's length boundary."""
+    w = WORKLOADS["bf16_varlen"]
+    tensors, outs, lengths = _run_workload(w)
+    nb = w.n // BLOCK
+    for bh in [(0, 0), (1, 5), (3, 11)]:
+        _check_window(w, tensors, outs, bh, 0, nb, lengths)
+    rng = np.random.default_rng(0)
+    for b in range(w.batch):
+        Lb = int(lengths[b])
+        edge = (Lb - 1) // BLOCK
+        h = int(rng.integers(w.heads))
+        _check_window(w, tensors, outs, (b, h), max(0, edge - 3), min(nb, edge + 4), lengths)
+    for t in outs:
+        for b in range(w.batch):
+            Lb = int(lengths[b])
+            assert (t[b, :, Lb:] == 0).all() or torch.isneginf(t[b, :, Lb:]).all()
+
+
+def test_bf16_n131k_workload():
+    """bf16, 1 x 16 x 131072 x 128, R = 4: sampled windows incl. both ends."""
+    w = WORKLOADS["bf16_n131k"]
+    tensors, outs, lengths = _run_workload(w)
+    nb = w.n // BLOCK
+    rng = np.random.default_rng(1)
+    for h, lo in [(0, 0), (15, nb - 12), (7, 2000)] + [
+            (int(rng.integers(16)), int(rng.integers(0, nb - 12))) for _ in range(3)]:
+        _check_window(w, tensors, outs, (0, h), lo, lo + 12, lengths)
+
+
+def test_bf16_n1m_workload():
+    """bf16, 1 x 8 x 1048576 x 64, R = 8: sampled windows; peak memory linear in n."""
+    w = WORKLOADS["bf16_n1m"]
+    torch.cuda.reset_peak_memory_stats()
+    tensors, outs, lengths = _run_workload(w)
+    peak = torch.cuda.max_memory_allocated()
+    elems = w.batch * w.heads * w.n * w.d
+    # 9 bf16 tensors (q k v do o dq dk dv + slack), lse, D and the fp32 dQ accumulator
+    assert peak <= elems * 2 * 9 + elems * 4 + w.batch * w.heads * w.n * 8 + (64 << 20)
+    nb = w.n // BLOCK
+    rng = np.random.default_rng(2)
+    for h, lo in [(0, 0), (7, nb - 20)] + [
+            (int(rng.integers(8)), int(rng.integers(0, nb - 20))) for _ in range(3)]:
+        _check_window(w, tensors, outs, (0, h), lo, lo + 20, lengths)

@@ -122,6 +122,31 @@ NB_API nb_status nb_attn_bwd(const void* q, const void* k, const void* v, const 
                       int heads, int n, int d, int R, int dtype, void* stream);
 
 /*
+ * nb_attn_bwd_noalloc - nb_attn_bwd for callers that cannot allocate device
+ * memory.  The NucleoByte page has no counterpart: it exists for callers that
+ * cannot hand the library a workspace, such as a host program whose device
+ * memory is wholly owned by another allocator, an embedding through a
+ * foreign-function interface with no allocator, or a latency-critical loop in
+ * which cudaMalloc/cudaFree (which may synchronise the device) are not allowed.
+ * Same arguments, results and errors as nb_attn_bwd, minus the workspace: the
+ * scratch is a fixed array of NB_NOALLOC_SCRATCH_BYTES compiled into the
+ * library, held on every GPU where the library's code is loaded until the
+ * process exits.  Shapes whose nb_attn_bwd_workspace_size exceeds that limit
+ * return NB_ERR_WORKSPACE without launching.  This entry point allocates
+ * nothing.  Its first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture.  Every call shares the one array, so calls that overlap on the GPU
+ * (other streams or host threads) race and must be serialised by the caller;
+ * each call rewrites what it reads from the array, so an earlier call's
+ * leftover contents do not affect results.
+ */
+#define NB_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+NB_API nb_status nb_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                     const void* dout, const float* lse, const int32_t* lengths,
+                                     void* dq, void* dk, void* dv, int batch, int heads, int n,
+                                     int d, int R, int dtype, void* stream);
+
+/*
  * nb_tokenize_kmer - fused 2-bit DNA k-mer tokenizer.
  * (NucleoByte page, sections 1 "Token Blur", 2 "Fused 2-Bit Tokenization",
  * 5 "Architecture Size" and "Evaluation Output Verification".)

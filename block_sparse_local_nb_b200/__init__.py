@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     lib,
     nb_attn_bwd,
     nb_attn_fwd,
+    nb_kernel_error,
     nb_status_string,
     nb_tokenize_kmer,
 )

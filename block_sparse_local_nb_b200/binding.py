@@ -25,6 +25,7 @@ _I = ctypes.c_int
 _SIGS = [
     ("nb_status_string", ctypes.c_char_p, [_I]),
     ("nb_abi_version", _I, []),
+    ("nb_kernel_error", _I, [ctypes.POINTER(ctypes.c_int), _I]),
     ("nb_attn_fwd", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     ("nb_attn_bwd_workspace_size", ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     ("nb_attn_bwd", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
@@ -79,6 +80,13 @@ def _stream(stream):
 def _check(status: int, what: str):
     if status != 0:
         raise NbError(status, what)
+
+
+def nb_kernel_error(clear: bool = True) -> int:
+    """Synchronise the device and return the first recorded kernel wait-timeout code (0 = none)."""
+    code = ctypes.c_int(0)
+    _check(lib().nb_kernel_error(ctypes.byref(code), 1 if clear else 0), "nb_kernel_error")
+    return code.value
 
 
 def nb_status_string(status: int) -> str:

@@ -5,6 +5,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/nb.h"
 #include "nb_internal.h"
 
@@ -13,6 +15,27 @@ namespace {
 constexpr int kMaxDevices = 64;
 // Per-device cache: 0 = unknown, 1 = sm_100 (supported), -1 = other.
 int g_device_ok[kMaxDevices];
+
+// Device word where kernels record the first wait-timeout code (0 = none),
+// and its device address per device (looked up once).
+__device__ int g_kernel_error;
+std::mutex g_err_mutex;
+int* g_err_addr[kMaxDevices];
+
+int* error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_err_mutex);
+  if (g_err_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kernel_error) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_err_addr[dev] = static_cast<int*>(p);
+  }
+  return g_err_addr[dev];
+}
 
 nb_status check_device() {
   int dev = 0;
@@ -55,6 +78,7 @@ nb::AttnArgs make_args(const void* q, const void* k, const void* v, const void* 
   a.dq = dq; a.dk = dk; a.dv = dv; a.workspace = ws;
   a.batch = batch; a.heads = heads; a.n = n; a.d = d; a.R = R;
   a.scale = static_cast<float>(1.0 / sqrt(static_cast<double>(d)));
+  a.err = error_word();
   return a;
 }
 
@@ -77,6 +101,17 @@ const char* nb_status_string(int status) {
 
 int nb_abi_version(void) { return 100; }
 
+nb_status nb_kernel_error(int* code, int clear) {
+  if (!code) return NB_ERR_INVALID_ARG;
+  *code = 0;
+  int* w = error_word();
+  if (!w) return NB_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return NB_ERR_CUDA;
+  if (cudaMemcpy(code, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return NB_ERR_CUDA;
+  if (clear && *code != 0 && cudaMemset(w, 0, sizeof(int)) != cudaSuccess) return NB_ERR_CUDA;
+  return NB_OK;
+}
+
 nb_status nb_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                       const int32_t* lengths, int batch, int heads, int n, int d, int R,
                       int dtype, void* stream) {
@@ -92,7 +127,8 @@ nb_status nb_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   nb::AttnArgs a = make_args(q, k, v, o, nullptr, lse, lengths, nullptr, nullptr, nullptr,
                              nullptr, batch, heads, n, d, R);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = dtype == NB_F32 ? nb::launch_attn_fwd_f32(a, s) : nb::launch_attn_fwd_bf16(a, s);
+  cudaError_t e =
+      dtype == NB_F32 ? nb::launch_attn_fwd_f32(a, s) : nb::launch_attn_fwd_bf16_tc(a, s);
   return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
 }
 

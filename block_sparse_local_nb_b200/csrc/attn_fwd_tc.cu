@@ -1,0 +1,458 @@
+// Banded block-sparse local attention forward on the 5th-generation tensor
+// cores (tcgen05 + TMEM), bf16 in / fp32 accumulate.  (NucleoByte page,
+// section 3: band |i - j| <= R over blocks of B = 32, scores Q K^T / sqrt(d),
+// online softmax with running max, running sum and running output.)
+//
+// Work item = one query tile of 128 rows (four query blocks) of one (batch,
+// head).  The union of the four bands is the key-block window
+// [4t - R, 4t + 3 + R] (clipped to the sequence and its length), processed in
+// chunks of 128 keys (four key blocks).  A persistent grid of one CTA per SM
+// walks the items; consecutive CTAs take neighbouring tiles at the same time,
+// so the key/value blocks their windows share are served from L2.
+//
+// Warp roles (256 threads):
+//   warp 0     TMA producer: Q tile, then K and V chunks, into 128-byte
+//              swizzled shared memory (3-D tensor maps; rows outside [0, n)
+//              are zero-filled by TMA and masked).
+//   warp 1     TMEM owner and MMA issuer (one thread):
+//                S_c = Q K_c^T   (M 128, N 128, K d)   -> TMEM, two buffers
+//                O  += P_c V_c   (M 128, N d,   K 128) -> TMEM, two buffers
+//              S_{c+1} is issued before P_c V_c so the softmax of the next
+//              chunk overlaps the P V product.
+//   warps 4-7  softmax: thread r owns row r (TMEM lane r).  Per chunk it reads
+//              its 128 scores, masks keys outside its query block's band or
+//              past the length, updates the running max and sum (base 2), and
+//              writes P = 2^(s - m) as bf16 into shared memory for the P V
+//              product.  The running output lives in TMEM; it is rescaled
+//              (load, multiply, store) only when the row max grows by more
+//              than 2^8, otherwise the stale max is kept (P <= 2^8, exact after
+//              the final division).  Epilogue: O / l -> bf16, lse = m + log l.
+//   warps 2-3  idle.
+// Every mbarrier wait is bounded; on a timeout the kernel records an error
+// code in the caller-visible error word and tears down (frees TMEM) instead
+// of hanging.
+#include <math.h>
+
+#include "nb_internal.h"
+#include "sm100.cuh"
+#include "warp_mma.cuh"
+
+namespace nb {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 256;
+constexpr int kRows = 128;   // query rows per tile
+constexpr int kChunk = 128;  // keys per chunk
+constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 64 bf16
+constexpr float kTau = 8.0f;      // lazy-rescale threshold, log2 units
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D>
+struct Cfg {
+  static constexpr int NQ = D == 64 ? 2 : 1;   // Q tile buffers
+  static constexpr int NKV = D == 64 ? 3 : 2;  // K/V chunk stages
+  static constexpr int NP = 2;                 // P buffers
+  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kKBytes = kChunk * D * 2;
+  static constexpr int kPBytes = kRows * kChunk * 2;
+  static constexpr int oQ = 0;
+  static constexpr int oK = oQ + NQ * kQBytes;
+  static constexpr int oV = oK + NKV * kKBytes;
+  static constexpr int oP = oV + NKV * kKBytes;
+  static constexpr int oBar = oP + NP * kPBytes;
+  // barrier indices
+  static constexpr int bQFull = 0, bQFree = bQFull + NQ, bKVFull = bQFree + NQ,
+                       bKVFree = bKVFull + NKV, bSFull = bKVFree + NKV, bSFree = bSFull + 2,
+                       bPFull = bSFree + 2, bPFree = bPFull + NP, bOFull = bPFree + NP,
+                       bOFree = bOFull + 2, bDone = bOFree + 2, nBar = bDone + 1;
+  static constexpr int oSlot = oBar + nBar * 8;
+  static constexpr int kSmem = oSlot + 16 + 1024;  // + slack for 1024-byte alignment
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t tS = 0;    // S buffers: columns [0,128) and [128,256)
+  static constexpr uint32_t tO = 256;  // O buffers: [256, 256+D) and [256+D, 256+2D)
+};
+
+struct Params {
+  AttnArgs a;
+  int ntiles;  // query tiles per (batch, head)
+  int items;   // batch * heads * ntiles
+};
+
+struct Item {
+  int b, h, tile, L, J0, nch;
+};
+
+__device__ __forceinline__ Item decode(const Params& p, int it) {
+  const AttnArgs& a = p.a;
+  Item x;
+  const int bh = it / p.ntiles;
+  x.tile = it - bh * p.ntiles;
+  x.b = bh / a.heads;
+  x.h = bh - x.b * a.heads;
+  int L = a.lengths ? a.lengths[x.b] : a.n;
+  x.L = min(max(L, 0), a.n);
+  const int nb = a.n / kBlock;
+  x.J0 = 0;
+  x.nch = 0;
+  if (x.tile * kRows < x.L) {
+    const int qb_last = min(x.tile * 4 + 3, nb - 1);
+    x.J0 = max(0, x.tile * 4 - a.R);
+    const int J1 = min(min(qb_last + a.R, nb - 1), (x.L - 1) / kBlock);
+    x.nch = (J1 - x.J0 + 4) / 4;
+  }
+  return x;
+}
+
+// error codes: 0x10 + site
+enum : int { kErrQFree = 0x11, kErrKVFree, kErrQFull, kErrKVFull, kErrSFree, kErrOFree, kErrPFull,
+             kErrSFull, kErrPFree, kErrPPrev, kErrOFull, kErrDone };
+
+template <int D>
+__device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tq,
+                        const CUtensorMap* tk, const CUtensorMap* tv) {
+  using C = Cfg<D>;
+  const uint32_t bar = base + C::oBar;
+  int g = 0, tc = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const Item x = decode(p, it);
+    if (x.nch == 0) continue;
+    const int bh = x.b * p.a.heads + x.h;
+    const int qs = tc % C::NQ;
+    if (!mbar_wait(bar + 8 * (C::bQFree + qs), ((tc / C::NQ) & 1) ^ 1)) return kErrQFree;
+    mbar_arrive_expect_tx(bar + 8 * (C::bQFull + qs), C::kQBytes);
+#pragma unroll
+    for (int s = 0; s < D / 64; ++s)
+      tma_load_3d(base + C::oQ + qs * C::kQBytes + s * kSlab, tq, bar + 8 * (C::bQFull + qs),
+                  s * 64, x.tile * kRows, bh);
+    for (int c = 0; c < x.nch; ++c) {
+      const int G = g + c, st = G % C::NKV;
+      if (!mbar_wait(bar + 8 * (C::bKVFree + st), ((G / C::NKV) & 1) ^ 1)) return kErrKVFree;
+      const uint32_t full = bar + 8 * (C::bKVFull + st);
+      mbar_arrive_expect_tx(full, 2 * C::kKBytes);
+      const int y = (x.J0 + 4 * c) * kBlock;
+#pragma unroll
+      for (int s = 0; s < D / 64; ++s) {
+        tma_load_3d(base + C::oK + st * C::kKBytes + s * kSlab, tk, full, s * 64, y, bh);
+        tma_load_3d(base + C::oV + st * C::kKBytes + s * kSlab, tv, full, s * 64, y, bh);
+      }
+    }
+    g += x.nch;
+    ++tc;
+  }
+  return 0;
+}
+
+template <int D>
+__device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
+  using C = Cfg<D>;
+  const uint32_t bar = base + C::oBar;
+  constexpr uint32_t kIdS = idesc_bf16_f32(128, kChunk, false, false);  // Q K^T: both K-major
+  constexpr uint32_t kIdPV = idesc_bf16_f32(128, 64, false, true);      // P V: V is MN-major
+  int g = 0, tc = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const Item x = decode(p, it);
+    if (x.nch == 0) continue;
+    const int qs = tc % C::NQ, ob = tc % 2;
+    if (!mbar_wait(bar + 8 * (C::bQFull + qs), (tc / C::NQ) & 1)) return kErrQFull;
+    const uint32_t sQ = base + C::oQ + qs * C::kQBytes;
+    auto issue_s = [&](int c) -> int {
+      const int G = g + c, st = G % C::NKV, sb = G % 2;
+      if (!mbar_wait(bar + 8 * (C::bKVFull + st), (G / C::NKV) & 1)) return kErrKVFull;
+      if (!mbar_wait(bar + 8 * (C::bSFree + sb), ((G / 2) & 1) ^ 1)) return kErrSFree;
+      tc_fence_after();
+      const uint32_t sK = base + C::oK + st * C::kKBytes;
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
+        mma_bf16_ss(tmem + C::tS + sb * kChunk, smem_desc_sw128(sQ + off, 0, 1024),
+                    smem_desc_sw128(sK + off, 0, 1024), kIdS, k > 0);
+      }
+      mma_commit(bar + 8 * (C::bSFull + sb));
+      return 0;
+    };
+    int e = issue_s(0);
+    if (e) return e;
+    for (int c = 0; c < x.nch; ++c) {
+      if (c + 1 < x.nch) {
+        if ((e = issue_s(c + 1))) return e;
+      } else {
+        mma_commit(bar + 8 * (C::bQFree + qs));  // all S products of this tile issued
+      }
+      const int G = g + c, st = G % C::NKV, pb = G % C::NP;
+      if (c == 0 && !mbar_wait(bar + 8 * (C::bOFree + ob), ((tc / 2) & 1) ^ 1)) return kErrOFree;
+      if (!mbar_wait(bar + 8 * (C::bPFull + pb), (G / C::NP) & 1)) return kErrPFull;
+      tc_fence_after();
+      const uint32_t sP = base + C::oP + pb * C::kPBytes;
+      const uint32_t sV = base + C::oV + st * C::kKBytes;
+#pragma unroll
+      for (int k = 0; k < kChunk / 16; ++k) {
+        const uint64_t ad = smem_desc_sw128(sP + (k >> 2) * kSlab + (k & 3) * 32, 0, 1024);
+#pragma unroll
+        for (int s = 0; s < D / 64; ++s)  // one N = 64 product per 64-column slab of V
+          mma_bf16_ss(tmem + C::tO + ob * D + s * 64, ad,
+                      smem_desc_sw128(sV + s * kSlab + k * 2048, 1024, 1024), kIdPV,
+                      c > 0 || k > 0);
+      }
+      mma_commit(bar + 8 * (C::bKVFree + st));
+      mma_commit(bar + 8 * (C::bPFree + pb));
+      if (c == x.nch - 1) mma_commit(bar + 8 * (C::bOFull + ob));
+    }
+    g += x.nch;
+    ++tc;
+  }
+  return 0;
+}
+
+template <int D>
+__device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, uint32_t tmem,
+                                int wq, int lane) {
+  using C = Cfg<D>;
+  const AttnArgs& a = p.a;
+  const uint32_t bar = base + C::oBar;
+  const int r = wq * 32 + lane;  // tile row == TMEM lane
+  const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const int nb = a.n / kBlock;
+  const float sl2 = a.scale * kLog2e;
+  auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
+  int g = 0, tc = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const Item x = decode(p, it);
+    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
+    const int q = x.tile * kRows + r;
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) + (bh * a.n + q) * D;
+    if (x.nch == 0) {  // the whole tile is padding
+      if (q < a.n) {
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) reinterpret_cast<uint4*>(orow)[i] = make_uint4(0, 0, 0, 0);
+        if (a.lse) a.lse[bh * a.n + q] = -INFINITY;
+      }
+      continue;
+    }
+    const int qb = q / kBlock;
+    const bool row_valid = q < x.L;
+    float m_used = -INFINITY, l = 0.f;
+    for (int c = 0; c < x.nch; ++c) {
+      const int G = g + c, sb = G % 2, pb = G % C::NP;
+      if (!all_ok(mbar_wait(bar + 8 * (C::bSFull + sb), (G / 2) & 1))) return kErrSFull;
+      tc_fence_after();
+      float s[4][32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tmem_ld32(trow + C::tS + sb * kChunk + 32 * j, s[j]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) reg_fence(s[j]);
+      tc_fence_before();
+      mbar_arrive(bar + 8 * (C::bSFree + sb));
+
+      bool vis[4];
+      float cmax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int kb = x.J0 + 4 * c + j;
+        vis[j] = row_valid && kb < nb && abs(kb - qb) <= a.R && kb * kBlock < x.L;
+        if (vis[j]) {
+          const int lim = x.L - kb * kBlock;  // keys at or past the length are masked
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float v = i < lim ? s[j][i] * sl2 : -INFINITY;
+            s[j][i] = v;
+            cmax = fmaxf(cmax, v);
+          }
+        }
+      }
+      bool need = false;
+      float alpha = 1.f;
+      if (cmax > m_used + kTau) {
+        if (m_used != -INFINITY) {
+          need = true;
+          alpha = exp2f(m_used - cmax);
+        }
+        m_used = cmax;
+      }
+      if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + pb), ((G / C::NP) & 1) ^ 1))) return kErrPFree;
+      if (__any_sync(0xffffffffu, need)) {
+        // the previous P V product of this tile must have landed before O is rescaled
+        const int Gp = G - 1;
+        if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + Gp % C::NP), (Gp / C::NP) & 1)))
+          return kErrPPrev;
+        tc_fence_after();
+        const uint32_t to = trow + C::tO + (tc % 2) * D;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          float ov[32];
+          tmem_ld32(to + 32 * j, ov);
+          tmem_wait_ld();
+          reg_fence(ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+          tmem_st32(to + 32 * j, ov);
+        }
+        tmem_wait_st();
+        l *= alpha;
+      }
+      // P = 2^(s - m) in bf16, row r of the 128-byte-swizzled P tile
+      uint8_t* prow = gbase + C::oP + pb * C::kPBytes + r * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int chunk = 4 * j + cc;  // 8 keys per 16-byte chunk
+          uint32_t w[4];
+          if (vis[j]) {
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+              const float p0 = exp2f(s[j][8 * cc + 2 * e2] - m_used);
+              const float p1 = exp2f(s[j][8 * cc + 2 * e2 + 1] - m_used);
+              l += p0 + p1;
+              w[e2] = pack_bf16(p0, p1);
+            }
+          } else {
+            w[0] = w[1] = w[2] = w[3] = 0u;
+          }
+          const int slab = chunk >> 3, c8 = chunk & 7;
+          *reinterpret_cast<uint4*>(prow + slab * kSlab + ((c8 ^ (r & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar + 8 * (C::bPFull + pb));
+    }
+    // epilogue: O / l
+    const int ob = tc % 2;
+    if (!all_ok(mbar_wait(bar + 8 * (C::bOFull + ob), (tc / 2) & 1))) return kErrOFull;
+    tc_fence_after();
+    float o[D / 32][32];
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) tmem_ld32(trow + C::tO + ob * D + 32 * j, o[j]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) reg_fence(o[j]);
+    tc_fence_before();
+    mbar_arrive(bar + 8 * (C::bOFree + ob));
+    const bool has = row_valid && l > 0.f;
+    const float inv = has ? 1.f / l : 0.f;
+    if (q < a.n) {
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 u;
+          u.x = pack_bf16(o[j][8 * v + 0] * inv, o[j][8 * v + 1] * inv);
+          u.y = pack_bf16(o[j][8 * v + 2] * inv, o[j][8 * v + 3] * inv);
+          u.z = pack_bf16(o[j][8 * v + 4] * inv, o[j][8 * v + 5] * inv);
+          u.w = pack_bf16(o[j][8 * v + 6] * inv, o[j][8 * v + 7] * inv);
+          reinterpret_cast<uint4*>(orow)[4 * j + v] = u;
+        }
+      }
+      if (a.lse) a.lse[bh * a.n + q] = has ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+    }
+    g += x.nch;
+    ++tc;
+  }
+  return 0;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bar = base + C::oBar;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NQ; ++i) {
+      mbar_init(bar + 8 * (C::bQFull + i), 1);
+      mbar_init(bar + 8 * (C::bQFree + i), 1);
+    }
+    for (int i = 0; i < C::NKV; ++i) {
+      mbar_init(bar + 8 * (C::bKVFull + i), 1);
+      mbar_init(bar + 8 * (C::bKVFree + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar + 8 * (C::bSFull + i), 1);
+      mbar_init(bar + 8 * (C::bSFree + i), 128);
+      mbar_init(bar + 8 * (C::bOFull + i), 1);
+      mbar_init(bar + 8 * (C::bOFree + i), 128);
+    }
+    for (int i = 0; i < C::NP; ++i) {
+      mbar_init(bar + 8 * (C::bPFull + i), 128);
+      mbar_init(bar + 8 * (C::bPFree + i), 1);
+    }
+    mbar_init(bar + 8 * C::bDone, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tq);
+    prefetch_tmap(&tk);
+    prefetch_tmap(&tv);
+  }
+  if (warp == 1) {
+    tmem_alloc(base + C::oSlot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + C::oSlot);
+
+  int err = 0;
+  if (warp == 0) {
+    if (lane == 0) err = producer<D>(p, base, &tq, &tk, &tv);
+  } else if (warp == 1) {
+    if (lane == 0) err = mma_issuer<D>(p, base, tmem);
+  } else if (warp >= 4) {
+    err = softmax_epilogue<D>(p, base, gbase, tmem, warp - 4, lane);
+  }
+  if (err) record_error(p.a.err, err);
+
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) {  // every tensor-core operation of this CTA has completed
+      mma_commit(bar + 8 * C::bDone);
+      if (!mbar_wait(bar + 8 * C::bDone, 0)) record_error(p.a.err, kErrDone);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
+  using C = Cfg<D>;
+  const int64_t heads_total = static_cast<int64_t>(a.batch) * a.heads;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_bf16_rows(&tq, a.q, D, a.n, heads_total, kRows) ||
+      !make_tmap_bf16_rows(&tk, a.k, D, a.n, heads_total, kChunk) ||
+      !make_tmap_bf16_rows(&tv, a.v, D, a.n, heads_total, kChunk))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.a = a;
+  p.ntiles = (a.n + kRows - 1) / kRows;
+  const int64_t items = heads_total * p.ntiles;
+  if (items > (1ll << 30)) return cudaErrorInvalidValue;
+  p.items = static_cast<int>(items);
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  attn_fwd_tc_kernel<D><<<grid, kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t stream) {
+  return a.d == 64 ? launch<64>(a, stream) : launch<128>(a, stream);
+}
+
+}  // namespace nb

@@ -1,6 +1,7 @@
 // Internal declarations shared by the C-ABI layer and the kernel launchers.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -21,6 +22,7 @@ struct AttnArgs {
   void* dk;
   void* dv;
   void* workspace;
+  int* err;           // device word receiving the first wait-timeout code (may be null)
   int batch, heads, n, d, R;
   float scale;        // 1/sqrt(d)
 };
@@ -29,10 +31,16 @@ struct AttnArgs {
 size_t bwd_workspace_bytes(int64_t rows, int d);
 __host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
+// TMA map over a [heads_total][n][d] bf16 tensor with 128-byte swizzle and a
+// box of 64 columns x box_rows rows.
+bool make_tmap_bf16_rows(CUtensorMap* m, const void* base, int d, int64_t n, int64_t heads_total,
+                         int box_rows);
+int num_sms();  // SM count of the current device (cached)
+
 cudaError_t launch_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
                                  int k, cudaStream_t stream);
 cudaError_t launch_attn_fwd_f32(const AttnArgs& a, cudaStream_t stream);
-cudaError_t launch_attn_fwd_bf16(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_bwd_bf16(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace nb

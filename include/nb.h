@@ -18,8 +18,10 @@
  *
  * Conventions shared by every call:
  *   - Every pointer argument is a DEVICE pointer unless stated otherwise.  The
- *     caller owns every buffer; the library keeps no state between calls except
- *     a per-device cache of device properties, and allocates no device memory.
+ *     caller owns every buffer; the library allocates no device memory and
+ *     keeps no state between calls except per-device caches (device
+ *     properties, symbol addresses) and the kernel error word read by
+ *     nb_kernel_error.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream).  Arguments are validated on the host first: an invalid
  *     call returns a negative nb_status and launches nothing.  A failed launch
@@ -73,6 +75,16 @@ NB_API const char* nb_status_string(int status);
 
 /* ABI version of this library (major * 100 + minor). */
 NB_API int nb_abi_version(void);
+
+/*
+ * nb_kernel_error - report whether a kernel gave up waiting.  Every wait inside
+ * the tensor-core kernels is bounded (2 s); a kernel that runs out records a
+ * non-zero site code in a device word, frees its tensor memory and returns, so
+ * the context stays usable (its outputs are then undefined).  This call
+ * synchronises the current device, stores the recorded code (0 = none) in
+ * *code and, when `clear` is non-zero, resets it.
+ */
+NB_API nb_status nb_kernel_error(int* code, int clear);
 
 /*
  * nb_attn_fwd - banded block-sparse local attention, forward.

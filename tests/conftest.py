@@ -27,3 +27,15 @@ def read_golden(name):
             line = line.strip()
             if line and not line.startswith("#"):
                 yield line.split()
+
+
+@pytest.fixture(autouse=True)
+def _no_kernel_wait_timeouts(request):
+    """After every GPU test: no kernel gave up on a bounded wait."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import block_sparse_local_nb_b200 as nb
+
+    code = nb.nb_kernel_error(clear=True)
+    assert code == 0, f"a kernel recorded wait-timeout code {code:#x}"

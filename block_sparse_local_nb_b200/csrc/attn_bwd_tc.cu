@@ -1,0 +1,468 @@
+// Banded block-sparse local attention backward, main kernel, on the
+// 5th-generation tensor cores (tcgen05 + TMEM), bf16 in / fp32 accumulate.
+// (NucleoByte page, section 3 "Custom Backpropagation": P recomputed from the
+// stored log-sum-exp, D_i = sum_k dO_ik O_ik, dS = P (dO V^T - D); gradients of
+// shared key/value blocks accumulated with atomic adds.)
+//
+// Work item = one key tile of 128 keys (four key blocks) of one (batch, head).
+// The band is symmetric, so its dK and dV need only the query blocks
+// [4t - R, 4t + 3 + R], taken in chunks of 128 queries.  Per chunk, with keys
+// on the TMEM lanes (M = 128):
+//   S^T  = K Q^T          dP^T = V dO^T                       (N 128, K d)
+//   P^T  = 2^(S^T scale log2e - lse log2e),  dS^T = P^T (dP^T - D)   (CUDA cores)
+//   dV  += P^T dO         dK  += dS^T Q                        (N d, K 128)
+//   dQ_c = dS K           (queries on the lanes: dS^T read as an MN-major A)
+// dK and dV accumulate in TMEM over the item's chunks (deterministic); dQ_c is
+// added into an fp32 accumulator in global memory with a TMA bulk reduce-add.
+//
+// Warp roles (448 threads): warp 0 TMA producer (K, V tiles; Q, dO chunks;
+// the chunk's lse and D rows by bulk copy); warp 1 TMEM owner and MMA issuer;
+// warps 2-9 gradient warps: two groups of four, one per half of the chunk's
+// query columns, thread = key row; they also write dK (first group) and dV
+// (second group) at the end of an item; warps 10-13 dQ warps: thread = query
+// row, stage dQ_c in shared memory (reusing the chunk's Q/dO buffer) and
+// reduce it into global memory.  All waits are bounded (see sm100.cuh).
+#include <math.h>
+
+#include "nb_internal.h"
+#include "sm100.cuh"
+#include "warp_mma.cuh"
+
+namespace nb {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 448;
+constexpr int kRows = 128;        // keys per item, queries per chunk
+constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 128 bytes
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct Cfg {
+  static constexpr int NS = D == 64 ? 2 : 1;  // Q/dO chunk stages
+  static constexpr int kTile = kRows * D * 2;  // one [128 x D] bf16 tile
+  static constexpr int kPT = kRows * kRows * 2;  // one [128 x 128] bf16 tile
+  static constexpr int oK = 0;
+  static constexpr int oV = oK + kTile;
+  static constexpr int oQ = oV + kTile;  // stage s: Q at oQ + 2 s kTile, dO right after
+  static constexpr int oP = oQ + NS * 2 * kTile;
+  static constexpr int oDS = oP + kPT;
+  static constexpr int oLD = oDS + kPT;  // stage s: -lse log2e [128] then D [128], fp32
+  static constexpr int oBar = oLD + NS * 1024;
+  static constexpr int bKVFull = 0, bKVFree = 1, bQDFull = 2, bQDFree = bQDFull + NS,
+                       bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1, bPDSFull = bSDPFree + 1,
+                       bPDSFree = bPDSFull + 1, bDQFull = bPDSFree + 1, bDQFree = bDQFull + 1,
+                       bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1, bDone = bDKVFree + 1,
+                       nBar = bDone + 1;
+  static constexpr int oSlot = oBar + nBar * 8;
+  static constexpr int kSmem = oSlot + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D;
+  static constexpr uint32_t tDQ = D == 64 ? 384 : 0;  // for D = 128, dQ reuses the S columns
+};
+
+struct Params {
+  AttnArgs a;
+  BwdWorkspace ws;
+  int ntiles;  // key tiles per (batch, head)
+  int items;
+};
+
+struct Item {
+  int b, h, tile, L, I0, nch;
+};
+
+__device__ __forceinline__ Item decode(const Params& p, int it) {
+  const AttnArgs& a = p.a;
+  Item x;
+  const int bh = it / p.ntiles;
+  x.tile = it - bh * p.ntiles;
+  x.b = bh / a.heads;
+  x.h = bh - x.b * a.heads;
+  int L = a.lengths ? a.lengths[x.b] : a.n;
+  x.L = min(max(L, 0), a.n);
+  const int nb = a.n / kBlock;
+  x.I0 = 0;
+  x.nch = 0;
+  if (x.tile * kRows < x.L) {
+    const int kb_last = min(x.tile * 4 + 3, nb - 1);
+    x.I0 = max(0, x.tile * 4 - a.R);
+    const int I1 = min(min(kb_last + a.R, nb - 1), (x.L - 1) / kBlock);
+    x.nch = (I1 - x.I0 + 4) / 4;
+  }
+  return x;
+}
+
+enum : int { kErrKVFree = 0x31, kErrQDFree, kErrKVFull, kErrQDFull, kErrSDPFree, kErrDQFree,
+             kErrPDSFull, kErrDKVFree, kErrGQD, kErrSDPFull, kErrPDSFree, kErrDKVFull,
+             kErrDQFull, kErrDone };
+
+template <int D>
+__device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tk,
+                        const CUtensorMap* tv, const CUtensorMap* tq, const CUtensorMap* tdo) {
+  using C = Cfg<D>;
+  const AttnArgs& a = p.a;
+  const uint32_t bar = base + C::oBar;
+  int g = 0, tc = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const Item x = decode(p, it);
+    if (x.nch == 0) continue;
+    const int bh = x.b * a.heads + x.h;
+    if (!mbar_wait(bar + 8 * C::bKVFree, (tc & 1) ^ 1)) return kErrKVFree;
+    mbar_arrive_expect_tx(bar + 8 * C::bKVFull, 2 * C::kTile);
+#pragma unroll
+    for (int s = 0; s < D / 64; ++s) {
+      tma_load_3d(base + C::oK + s * kSlab, tk, bar + 8 * C::bKVFull, s * 64, x.tile * kRows, bh);
+      tma_load_3d(base + C::oV + s * kSlab, tv, bar + 8 * C::bKVFull, s * 64, x.tile * kRows, bh);
+    }
+    for (int c = 0; c < x.nch; ++c) {
+      const int G = g + c, st = G % C::NS;
+      if (!mbar_wait(bar + 8 * (C::bQDFree + st), ((G / C::NS) & 1) ^ 1)) return kErrQDFree;
+      const int q0 = (x.I0 + 4 * c) * kBlock;
+      const int rows = min(kRows, a.n - q0);  // lse / D rows that exist
+      const uint32_t full = bar + 8 * (C::bQDFull + st);
+      mbar_arrive_expect_tx(full, 2 * C::kTile + 8 * rows);
+      const uint32_t sq = base + C::oQ + st * 2 * C::kTile;
+#pragma unroll
+      for (int s = 0; s < D / 64; ++s) {
+        tma_load_3d(sq + s * kSlab, tq, full, s * 64, q0, bh);
+        tma_load_3d(sq + C::kTile + s * kSlab, tdo, full, s * 64, q0, bh);
+      }
+      const int64_t row0 = static_cast<int64_t>(bh) * a.n + q0;
+      const uint32_t sld = base + C::oLD + st * 1024;
+      bulk_load(sld, p.ws.nlse2 + row0, 4 * rows, full);
+      bulk_load(sld + 512, p.ws.D + row0, 4 * rows, full);
+    }
+    g += x.nch;
+    ++tc;
+  }
+  return 0;
+}
+
+template <int D>
+__device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
+  using C = Cfg<D>;
+  const uint32_t bar = base + C::oBar;
+  constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // K Q^T, V dO^T
+  constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, false, true);    // P^T dO, dS^T Q
+  constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, true, true);      // dS K
+  const uint32_t sK = base + C::oK, sV = base + C::oV, sP = base + C::oP, sS = base + C::oDS;
+  int g = 0, tc = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const Item x = decode(p, it);
+    if (x.nch == 0) continue;
+    if (!mbar_wait(bar + 8 * C::bKVFull, tc & 1)) return kErrKVFull;
+    for (int c = 0; c < x.nch; ++c) {
+      const int G = g + c, st = G % C::NS;
+      const uint32_t sQ = base + C::oQ + st * 2 * C::kTile, sdO = sQ + C::kTile;
+      if (!mbar_wait(bar + 8 * (C::bQDFull + st), (G / C::NS) & 1)) return kErrQDFull;
+      if (!mbar_wait(bar + 8 * C::bSDPFree, (G & 1) ^ 1)) return kErrSDPFree;
+      if (D == 128 && !mbar_wait(bar + 8 * C::bDQFree, (G & 1) ^ 1)) return kErrDQFree;
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
+        mma_bf16_ss(tmem + C::tS, smem_desc_sw128(sK + off, 0, 1024),
+                    smem_desc_sw128(sQ + off, 0, 1024), kIdS, k > 0);
+        mma_bf16_ss(tmem + C::tDP, smem_desc_sw128(sV + off, 0, 1024),
+                    smem_desc_sw128(sdO + off, 0, 1024), kIdS, k > 0);
+      }
+      mma_commit(bar + 8 * C::bSDPFull);
+      if (!mbar_wait(bar + 8 * C::bPDSFull, G & 1)) return kErrPDSFull;
+      if (c == 0 && !mbar_wait(bar + 8 * C::bDKVFree, (tc & 1) ^ 1)) return kErrDKVFree;
+      if (D == 64 && !mbar_wait(bar + 8 * C::bDQFree, (G & 1) ^ 1)) return kErrDQFree;
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < kRows / 16; ++k) {  // k over the chunk's queries
+        const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
+        mma_bf16_ss(tmem + C::tDV, smem_desc_sw128(sP + off, 0, 1024),
+                    smem_desc_sw128(sdO + k * 2048, kSlab, 1024), kIdKV, c > 0 || k > 0);
+        mma_bf16_ss(tmem + C::tDK, smem_desc_sw128(sS + off, 0, 1024),
+                    smem_desc_sw128(sQ + k * 2048, kSlab, 1024), kIdKV, c > 0 || k > 0);
+      }
+#pragma unroll
+      for (int k = 0; k < kRows / 16; ++k)  // k over the tile's keys
+        mma_bf16_ss(tmem + C::tDQ, smem_desc_sw128(sS + k * 2048, kSlab, 1024),
+                    smem_desc_sw128(sK + k * 2048, kSlab, 1024), kIdQ, k > 0);
+      mma_commit(bar + 8 * C::bPDSFree);
+      mma_commit(bar + 8 * C::bDQFull);
+    }
+    mma_commit(bar + 8 * C::bDKVFull);
+    mma_commit(bar + 8 * C::bKVFree);
+    g += x.nch;
+    ++tc;
+  }
+  return 0;
+}
+
+// Gradient warps: thread = key row r; half hf owns query columns [64 hf, 64 hf + 64).
+template <int D>
+__device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32_t tmem, int wq,
+                          int hf, int lane) {
+  using C = Cfg<D>;
+  const AttnArgs& a = p.a;
+  const uint32_t bar = base + C::oBar;
+  const int r = wq * 32 + lane;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const int nb = a.n / kBlock;
+  const float sl2 = a.scale * kLog2e;
+  auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
+  int g = 0, tc = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const Item x = decode(p, it);
+    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
+    const int k = x.tile * kRows + r;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(hf == 0 ? a.dk : a.dv) + (bh * a.n + k) * D;
+    if (x.nch == 0) {  // every key of the tile is padding
+      if (k < a.n) {
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) reinterpret_cast<uint4*>(out)[i] = make_uint4(0, 0, 0, 0);
+      }
+      continue;
+    }
+    const bool row_valid = k < x.L;
+    const int kb = k / kBlock;
+    for (int c = 0; c < x.nch; ++c) {
+      const int G = g + c, st = G % C::NS;
+      if (!all_ok(mbar_wait(bar + 8 * (C::bQDFull + st), (G / C::NS) & 1))) return kErrGQD;
+      if (!all_ok(mbar_wait(bar + 8 * C::bSDPFull, G & 1))) return kErrSDPFull;
+      if (!all_ok(mbar_wait(bar + 8 * C::bPDSFree, (G & 1) ^ 1))) return kErrPDSFree;
+      tc_fence_after();
+      const float* nl = reinterpret_cast<const float*>(gbase + C::oLD + st * 1024);
+      const float* Dv = nl + 128;
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int j = 2 * hf + jj;  // 32-query group within the chunk
+        float s[32], dp[32];
+        tmem_ld32(trow + C::tS + 32 * j, s);
+        tmem_ld32(trow + C::tDP + 32 * j, dp);
+        tmem_wait_ld();
+        reg_fence(s);
+        reg_fence(dp);
+        if (jj == 1) {
+          tc_fence_before();
+          mbar_arrive(bar + 8 * C::bSDPFree);
+        }
+        const int qb = x.I0 + 4 * c + j;
+        const bool vis = row_valid && qb < nb && abs(qb - kb) <= a.R;
+        uint8_t* prow = gbase + C::oP + hf * kSlab + r * 128;
+        uint8_t* srow = gbase + C::oDS + hf * kSlab + r * 128;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t wp[4], ws[4];
+          if (vis) {
+            const float4 n0 = *reinterpret_cast<const float4*>(nl + 32 * j + 8 * cc);
+            const float4 n1 = *reinterpret_cast<const float4*>(nl + 32 * j + 8 * cc + 4);
+            const float4 d0 = *reinterpret_cast<const float4*>(Dv + 32 * j + 8 * cc);
+            const float4 d1 = *reinterpret_cast<const float4*>(Dv + 32 * j + 8 * cc + 4);
+            const float nv[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+            const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+            float pe[8], de[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              pe[e] = exp2f(fmaf(s[8 * cc + e], sl2, nv[e]));  // -inf for padding queries -> 0
+              de[e] = pe[e] * (dp[8 * cc + e] - dv[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              wp[e] = pack_bf16(pe[2 * e], pe[2 * e + 1]);
+              ws[e] = pack_bf16(de[2 * e], de[2 * e + 1]);
+            }
+          } else {
+            wp[0] = wp[1] = wp[2] = wp[3] = 0u;
+            ws[0] = ws[1] = ws[2] = ws[3] = 0u;
+          }
+          const int ch = ((4 * jj + cc) ^ (r & 7)) << 4;
+          *reinterpret_cast<uint4*>(prow + ch) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
+          *reinterpret_cast<uint4*>(srow + ch) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar + 8 * C::bPDSFull);
+    }
+    // epilogue: first group writes dK (times 1/sqrt(d)), second group dV
+    if (!all_ok(mbar_wait(bar + 8 * C::bDKVFull, tc & 1))) return kErrDKVFull;
+    tc_fence_after();
+    const float mul = row_valid ? (hf == 0 ? a.scale : 1.f) : 0.f;
+    const uint32_t tsrc = trow + (hf == 0 ? C::tDK : C::tDV);
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) {
+      float v[32];
+      tmem_ld32(tsrc + 32 * j, v);
+      tmem_wait_ld();
+      reg_fence(v);
+      if (k < a.n) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          reinterpret_cast<uint4*>(out)[4 * j + u] =
+              make_uint4(pack_bf16(v[8 * u] * mul, v[8 * u + 1] * mul),
+                         pack_bf16(v[8 * u + 2] * mul, v[8 * u + 3] * mul),
+                         pack_bf16(v[8 * u + 4] * mul, v[8 * u + 5] * mul),
+                         pack_bf16(v[8 * u + 6] * mul, v[8 * u + 7] * mul));
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(bar + 8 * C::bDKVFree);
+    g += x.nch;
+    ++tc;
+  }
+  return 0;
+}
+
+// dQ warps: thread = query row r of the chunk.
+template <int D>
+__device__ int dq_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32_t tmem, int wq,
+                        int lane, const CUtensorMap* tdq) {
+  using C = Cfg<D>;
+  const AttnArgs& a = p.a;
+  const uint32_t bar = base + C::oBar;
+  const int r = wq * 32 + lane;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const bool leader = threadIdx.x == 10 * 32;
+  auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
+  int g = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const Item x = decode(p, it);
+    if (x.nch == 0) continue;
+    const int bh = x.b * a.heads + x.h;
+    for (int c = 0; c < x.nch; ++c) {
+      const int G = g + c, st = G % C::NS;
+      if (!all_ok(mbar_wait(bar + 8 * C::bDQFull, G & 1))) return kErrDQFull;
+      tc_fence_after();
+      // stage dQ_c (fp32) in the chunk's Q/dO buffer, laid out as D/32 swizzled boxes
+      uint8_t* stg = gbase + C::oQ + st * 2 * C::kTile;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        float v[32];
+        tmem_ld32(trow + C::tDQ + 32 * j, v);
+        tmem_wait_ld();
+        reg_fence(v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<float4*>(stg + j * kSlab + r * 128 + ((u ^ (r & 7)) << 4)) =
+              make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+      }
+      tc_fence_before();
+      mbar_arrive(bar + 8 * C::bDQFree);
+      fence_proxy_async_smem();
+      named_barrier(1, 128);
+      if (leader) {
+        const uint32_t sstg = base + C::oQ + st * 2 * C::kTile;
+        const int q0 = (x.I0 + 4 * c) * kBlock;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) tma_reduce_add_3d(tdq, sstg + j * kSlab, 32 * j, q0, bh);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(bar + 8 * (C::bQDFree + st));
+      }
+    }
+    g += x.nch;
+  }
+  return 0;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                       const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+                       const __grid_constant__ CUtensorMap tdq, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bar = base + C::oBar;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar + 8 * C::bKVFull, 1);
+    mbar_init(bar + 8 * C::bKVFree, 1);
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(bar + 8 * (C::bQDFull + i), 1);
+      mbar_init(bar + 8 * (C::bQDFree + i), 1);
+    }
+    mbar_init(bar + 8 * C::bSDPFull, 1);
+    mbar_init(bar + 8 * C::bSDPFree, 256);
+    mbar_init(bar + 8 * C::bPDSFull, 256);
+    mbar_init(bar + 8 * C::bPDSFree, 1);
+    mbar_init(bar + 8 * C::bDQFull, 1);
+    mbar_init(bar + 8 * C::bDQFree, 128);
+    mbar_init(bar + 8 * C::bDKVFull, 1);
+    mbar_init(bar + 8 * C::bDKVFree, 256);
+    mbar_init(bar + 8 * C::bDone, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tk);
+    prefetch_tmap(&tv);
+    prefetch_tmap(&tq);
+    prefetch_tmap(&tdo);
+    prefetch_tmap(&tdq);
+  }
+  if (warp == 1) {
+    tmem_alloc(base + C::oSlot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + C::oSlot);
+
+  int err = 0;
+  if (warp == 0) {
+    if (lane == 0) err = producer<D>(p, base, &tk, &tv, &tq, &tdo);
+  } else if (warp == 1) {
+    if (lane == 0) err = mma_issuer<D>(p, base, tmem);
+  } else if (warp < 10) {
+    err = grad_warps<D>(p, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane);
+  } else {
+    err = dq_warps<D>(p, base, gbase, tmem, warp & 3, lane, &tdq);
+  }
+  if (err) record_error(p.a.err, err);
+
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) {
+      mma_commit(bar + 8 * C::bDone);
+      if (!mbar_wait(bar + 8 * C::bDone, 0)) record_error(p.a.err, kErrDone);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
+  using C = Cfg<D>;
+  const int64_t heads_total = static_cast<int64_t>(a.batch) * a.heads;
+  Params p;
+  p.a = a;
+  p.ws = bwd_workspace(a.workspace, rows);
+  CUtensorMap tk, tv, tq, tdo, tdq;
+  if (!make_tmap_bf16_rows(&tk, a.k, D, a.n, heads_total, kRows) ||
+      !make_tmap_bf16_rows(&tv, a.v, D, a.n, heads_total, kRows) ||
+      !make_tmap_bf16_rows(&tq, a.q, D, a.n, heads_total, kRows) ||
+      !make_tmap_bf16_rows(&tdo, a.dout, D, a.n, heads_total, kRows) ||
+      !make_tmap_rows(&tdq, p.ws.dqacc, true, D, a.n, heads_total, 32, kRows))
+    return cudaErrorInvalidValue;
+  p.ntiles = (a.n + kRows - 1) / kRows;
+  const int64_t items = heads_total * p.ntiles;
+  if (items > (1ll << 30)) return cudaErrorInvalidValue;
+  p.items = static_cast<int>(items);
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
+  attn_bwd_tc_kernel<D><<<grid, kThreads, C::kSmem, stream>>>(tk, tv, tq, tdo, tdq, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_main_tc(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
+  return a.d == 64 ? launch<64>(a, rows, stream) : launch<128>(a, rows, stream);
+}
+
+}  // namespace nb

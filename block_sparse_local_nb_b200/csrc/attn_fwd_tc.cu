@@ -150,7 +150,7 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
   using C = Cfg<D>;
   const uint32_t bar = base + C::oBar;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, kChunk, false, false);  // Q K^T: both K-major
-  constexpr uint32_t kIdPV = idesc_bf16_f32(128, 64, false, true);      // P V: V is MN-major
+  constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);       // P V: V is MN-major
   int g = 0, tc = 0;
   for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
     const Item x = decode(p, it);
@@ -190,11 +190,9 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
 #pragma unroll
       for (int k = 0; k < kChunk / 16; ++k) {
         const uint64_t ad = smem_desc_sw128(sP + (k >> 2) * kSlab + (k & 3) * 32, 0, 1024);
-#pragma unroll
-        for (int s = 0; s < D / 64; ++s)  // one N = 64 product per 64-column slab of V
-          mma_bf16_ss(tmem + C::tO + ob * D + s * 64, ad,
-                      smem_desc_sw128(sV + s * kSlab + k * 2048, 1024, 1024), kIdPV,
-                      c > 0 || k > 0);
+        // V is MN-major: 64-column swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
+        mma_bf16_ss(tmem + C::tO + ob * D, ad, smem_desc_sw128(sV + k * 2048, kSlab, 1024), kIdPV,
+                    c > 0 || k > 0);
       }
       mma_commit(bar + 8 * (C::bKVFree + st));
       mma_commit(bar + 8 * (C::bPFree + pb));

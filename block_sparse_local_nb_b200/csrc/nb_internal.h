@@ -27,7 +27,6 @@ struct AttnArgs {
   float scale;        // 1/sqrt(d)
 };
 
-// Workspace layout of the backward: [row term D: rows fp32][dQ accumulator: rows*d fp32]
 size_t bwd_workspace_bytes(int64_t rows, int d);
 __host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
@@ -35,7 +34,28 @@ __host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + 
 // box of 64 columns x box_rows rows.
 bool make_tmap_bf16_rows(CUtensorMap* m, const void* base, int d, int64_t n, int64_t heads_total,
                          int box_rows);
+// Same for bf16 (box 64 columns) or fp32 tensors with a box of box_cols x box_rows
+// (box_cols * element size must be 128 bytes for the swizzle).
+bool make_tmap_rows(CUtensorMap* m, const void* base, bool f32, int d, int64_t n,
+                    int64_t heads_total, int box_cols, int box_rows);
 int num_sms();  // SM count of the current device (cached)
+
+// Backward workspace: [D: rows fp32][-lse*log2(e): rows fp32][dQ accumulator: rows*d fp32],
+// each region 256-byte aligned.
+struct BwdWorkspace {
+  float* D;
+  float* nlse2;
+  float* dqacc;
+};
+__host__ __device__ inline BwdWorkspace bwd_workspace(void* ws, int64_t rows) {
+  BwdWorkspace w;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  w.D = reinterpret_cast<float*>(p);
+  w.nlse2 = reinterpret_cast<float*>(p + align_up(rows * 4, 256));
+  w.dqacc = reinterpret_cast<float*>(p + 2 * align_up(rows * 4, 256));
+  return w;
+}
+cudaError_t launch_bwd_main_tc(const AttnArgs& a, int64_t rows, cudaStream_t stream);
 
 cudaError_t launch_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
                                  int k, cudaStream_t stream);

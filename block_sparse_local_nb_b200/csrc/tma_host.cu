@@ -31,19 +31,26 @@ int g_sms[kMaxDevices];
 
 }  // namespace
 
-bool make_tmap_bf16_rows(CUtensorMap* m, const void* base, int d, int64_t n, int64_t heads_total,
-                         int box_rows) {
+bool make_tmap_rows(CUtensorMap* m, const void* base, bool f32, int d, int64_t n,
+                    int64_t heads_total, int box_cols, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const cuuint64_t esz = f32 ? 4 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
                         static_cast<cuuint64_t>(heads_total)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(n) * d * 2};
-  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esz, static_cast<cuuint64_t>(n) * d * esz};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16_rows(CUtensorMap* m, const void* base, int d, int64_t n, int64_t heads_total,
+                         int box_rows) {
+  return make_tmap_rows(m, base, false, d, n, heads_total, 64, box_rows);
 }
 
 int num_sms() {

@@ -40,21 +40,25 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
-  static constexpr int NS = D == 64 ? 2 : 1;  // Q/dO chunk stages
+  // D = 64: K/V tiles double-buffered and S/dP of chunk G+1 issued before the
+  // dV/dK/dQ products of chunk G (the gradient warps of G+1 then overlap them).
+  // D = 128: TMEM is full (dQ reuses the S columns), so chunks run in order.
+  static constexpr bool kLook = D == 64;
+  static constexpr int NKV = D == 64 ? 2 : 1;  // K/V tile buffers
+  static constexpr int NS = D == 64 ? 2 : 1;   // Q/dO chunk stages
   static constexpr int kTile = kRows * D * 2;  // one [128 x D] bf16 tile
   static constexpr int kPT = kRows * kRows * 2;  // one [128 x 128] bf16 tile
-  static constexpr int oK = 0;
-  static constexpr int oV = oK + kTile;
-  static constexpr int oQ = oV + kTile;  // stage s: Q at oQ + 2 s kTile, dO right after
+  static constexpr int oK = 0;                   // buffer i: K at oK + 2 i kTile, V after it
+  static constexpr int oQ = NKV * 2 * kTile;     // stage s: Q at oQ + 2 s kTile, dO after it
   static constexpr int oP = oQ + NS * 2 * kTile;
   static constexpr int oDS = oP + kPT;
   static constexpr int oLD = oDS + kPT;  // stage s: -lse log2e [128] then D [128], fp32
   static constexpr int oBar = oLD + NS * 1024;
-  static constexpr int bKVFull = 0, bKVFree = 1, bQDFull = 2, bQDFree = bQDFull + NS,
-                       bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1, bPDSFull = bSDPFree + 1,
-                       bPDSFree = bPDSFull + 1, bDQFull = bPDSFree + 1, bDQFree = bDQFull + 1,
-                       bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1, bDone = bDKVFree + 1,
-                       nBar = bDone + 1;
+  static constexpr int bKVFull = 0, bKVFree = bKVFull + NKV, bQDFull = bKVFree + NKV,
+                       bQDFree = bQDFull + NS, bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1,
+                       bPDSFull = bSDPFree + 1, bPDSFree = bPDSFull + 1, bDQFull = bPDSFree + 1,
+                       bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
+                       bStg = bDKVFree + 1, bDone = bStg + 1, nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
   static constexpr int kSmem = oSlot + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
@@ -96,7 +100,7 @@ __device__ __forceinline__ Item decode(const Params& p, int it) {
 
 enum : int { kErrKVFree = 0x31, kErrQDFree, kErrKVFull, kErrQDFull, kErrSDPFree, kErrDQFree,
              kErrPDSFull, kErrDKVFree, kErrGQD, kErrSDPFull, kErrPDSFree, kErrDKVFull,
-             kErrDQFull, kErrDone };
+             kErrDQFull, kErrDone, kErrStg };
 
 template <int D>
 __device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tk,
@@ -109,12 +113,15 @@ __device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tk,
     const Item x = decode(p, it);
     if (x.nch == 0) continue;
     const int bh = x.b * a.heads + x.h;
-    if (!mbar_wait(bar + 8 * C::bKVFree, (tc & 1) ^ 1)) return kErrKVFree;
-    mbar_arrive_expect_tx(bar + 8 * C::bKVFull, 2 * C::kTile);
+    const int kvb = tc % C::NKV;
+    const uint32_t kvfull = bar + 8 * (C::bKVFull + kvb);
+    if (!mbar_wait(bar + 8 * (C::bKVFree + kvb), ((tc / C::NKV) & 1) ^ 1)) return kErrKVFree;
+    mbar_arrive_expect_tx(kvfull, 2 * C::kTile);
+    const uint32_t sk = base + C::oK + kvb * 2 * C::kTile;
 #pragma unroll
     for (int s = 0; s < D / 64; ++s) {
-      tma_load_3d(base + C::oK + s * kSlab, tk, bar + 8 * C::bKVFull, s * 64, x.tile * kRows, bh);
-      tma_load_3d(base + C::oV + s * kSlab, tv, bar + 8 * C::bKVFull, s * 64, x.tile * kRows, bh);
+      tma_load_3d(sk + s * kSlab, tk, kvfull, s * 64, x.tile * kRows, bh);
+      tma_load_3d(sk + C::kTile + s * kSlab, tv, kvfull, s * 64, x.tile * kRows, bh);
     }
     for (int c = 0; c < x.nch; ++c) {
       const int G = g + c, st = G % C::NS;
@@ -147,12 +154,47 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
   constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // K Q^T, V dO^T
   constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, false, true);    // P^T dO, dS^T Q
   constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, true, true);      // dS K
-  const uint32_t sK = base + C::oK, sV = base + C::oV, sP = base + C::oP, sS = base + C::oDS;
-  int g = 0, tc = 0;
+  const uint32_t sP = base + C::oP, sS = base + C::oDS;
+  // The chunk whose dV/dK/dQ products are still to be issued.
+  struct Pending {
+    bool valid;
+    int G, c, st, kvb, tc;
+    bool last;
+  } pend = {false, 0, 0, 0, 0, 0, false};
+  auto issue_grads = [&](const Pending& q) -> int {
+    const uint32_t sQ = base + C::oQ + q.st * 2 * C::kTile, sdO = sQ + C::kTile;
+    const uint32_t sK = base + C::oK + q.kvb * 2 * C::kTile;
+    if (!mbar_wait(bar + 8 * C::bPDSFull, q.G & 1)) return kErrPDSFull;
+    if (q.c == 0 && !mbar_wait(bar + 8 * C::bDKVFree, (q.tc & 1) ^ 1)) return kErrDKVFree;
+    if (D == 64 && !mbar_wait(bar + 8 * C::bDQFree, (q.G & 1) ^ 1)) return kErrDQFree;
+    tc_fence_after();
+#pragma unroll
+    for (int k = 0; k < kRows / 16; ++k) {  // k over the chunk's queries
+      const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
+      mma_bf16_ss(tmem + C::tDV, smem_desc_sw128(sP + off, 0, 1024),
+                  smem_desc_sw128(sdO + k * 2048, kSlab, 1024), kIdKV, q.c > 0 || k > 0);
+      mma_bf16_ss(tmem + C::tDK, smem_desc_sw128(sS + off, 0, 1024),
+                  smem_desc_sw128(sQ + k * 2048, kSlab, 1024), kIdKV, q.c > 0 || k > 0);
+    }
+#pragma unroll
+    for (int k = 0; k < kRows / 16; ++k)  // k over the tile's keys
+      mma_bf16_ss(tmem + C::tDQ, smem_desc_sw128(sS + k * 2048, kSlab, 1024),
+                  smem_desc_sw128(sK + k * 2048, kSlab, 1024), kIdQ, k > 0);
+    mma_commit(bar + 8 * C::bPDSFree);
+    mma_commit(bar + 8 * C::bDQFull);
+    if (q.last) {
+      mma_commit(bar + 8 * C::bDKVFull);
+      mma_commit(bar + 8 * (C::bKVFree + q.kvb));
+    }
+    return 0;
+  };
+  int g = 0, tc = 0, e = 0;
   for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
     const Item x = decode(p, it);
     if (x.nch == 0) continue;
-    if (!mbar_wait(bar + 8 * C::bKVFull, tc & 1)) return kErrKVFull;
+    const int kvb = tc % C::NKV;
+    const uint32_t sK = base + C::oK + kvb * 2 * C::kTile, sV = sK + C::kTile;
+    if (!mbar_wait(bar + 8 * (C::bKVFull + kvb), (tc / C::NKV) & 1)) return kErrKVFull;
     for (int c = 0; c < x.nch; ++c) {
       const int G = g + c, st = G % C::NS;
       const uint32_t sQ = base + C::oQ + st * 2 * C::kTile, sdO = sQ + C::kTile;
@@ -169,30 +211,18 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
                     smem_desc_sw128(sdO + off, 0, 1024), kIdS, k > 0);
       }
       mma_commit(bar + 8 * C::bSDPFull);
-      if (!mbar_wait(bar + 8 * C::bPDSFull, G & 1)) return kErrPDSFull;
-      if (c == 0 && !mbar_wait(bar + 8 * C::bDKVFree, (tc & 1) ^ 1)) return kErrDKVFree;
-      if (D == 64 && !mbar_wait(bar + 8 * C::bDQFree, (G & 1) ^ 1)) return kErrDQFree;
-      tc_fence_after();
-#pragma unroll
-      for (int k = 0; k < kRows / 16; ++k) {  // k over the chunk's queries
-        const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
-        mma_bf16_ss(tmem + C::tDV, smem_desc_sw128(sP + off, 0, 1024),
-                    smem_desc_sw128(sdO + k * 2048, kSlab, 1024), kIdKV, c > 0 || k > 0);
-        mma_bf16_ss(tmem + C::tDK, smem_desc_sw128(sS + off, 0, 1024),
-                    smem_desc_sw128(sQ + k * 2048, kSlab, 1024), kIdKV, c > 0 || k > 0);
+      const Pending cur = {true, G, c, st, kvb, tc, c == x.nch - 1};
+      if (C::kLook) {  // lookahead: chunk G-1's products go after S/dP of G
+        if (pend.valid && (e = issue_grads(pend))) return e;
+        pend = cur;
+      } else if ((e = issue_grads(cur))) {  // in order
+        return e;
       }
-#pragma unroll
-      for (int k = 0; k < kRows / 16; ++k)  // k over the tile's keys
-        mma_bf16_ss(tmem + C::tDQ, smem_desc_sw128(sS + k * 2048, kSlab, 1024),
-                    smem_desc_sw128(sK + k * 2048, kSlab, 1024), kIdQ, k > 0);
-      mma_commit(bar + 8 * C::bPDSFree);
-      mma_commit(bar + 8 * C::bDQFull);
     }
-    mma_commit(bar + 8 * C::bDKVFull);
-    mma_commit(bar + 8 * C::bKVFree);
     g += x.nch;
     ++tc;
   }
+  if (pend.valid && (e = issue_grads(pend))) return e;
   return 0;
 }
 
@@ -227,10 +257,10 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
       const int G = g + c, st = G % C::NS;
       if (!all_ok(mbar_wait(bar + 8 * (C::bQDFull + st), (G / C::NS) & 1))) return kErrGQD;
       if (!all_ok(mbar_wait(bar + 8 * C::bSDPFull, G & 1))) return kErrSDPFull;
-      if (!all_ok(mbar_wait(bar + 8 * C::bPDSFree, (G & 1) ^ 1))) return kErrPDSFree;
       tc_fence_after();
       const float* nl = reinterpret_cast<const float*>(gbase + C::oLD + st * 1024);
       const float* Dv = nl + 128;
+      uint32_t wp[2][16], ws[2][16];  // packed bf16 P^T and dS^T for this thread's 64 queries
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
         const int j = 2 * hf + jj;  // 32-query group within the chunk
@@ -240,17 +270,14 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
         tmem_wait_ld();
         reg_fence(s);
         reg_fence(dp);
-        if (jj == 1) {
+        if (jj == 1) {  // S and dP of this chunk are in registers: TMEM may be reused
           tc_fence_before();
           mbar_arrive(bar + 8 * C::bSDPFree);
         }
         const int qb = x.I0 + 4 * c + j;
         const bool vis = row_valid && qb < nb && abs(qb - kb) <= a.R;
-        uint8_t* prow = gbase + C::oP + hf * kSlab + r * 128;
-        uint8_t* srow = gbase + C::oDS + hf * kSlab + r * 128;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-          uint32_t wp[4], ws[4];
           if (vis) {
             const float4 n0 = *reinterpret_cast<const float4*>(nl + 32 * j + 8 * cc);
             const float4 n1 = *reinterpret_cast<const float4*>(nl + 32 * j + 8 * cc + 4);
@@ -261,23 +288,34 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
             float pe[8], de[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              pe[e] = exp2f(fmaf(s[8 * cc + e], sl2, nv[e]));  // -inf for padding queries -> 0
+              pe[e] = ex2_approx(fmaf(s[8 * cc + e], sl2, nv[e]));  // -inf for padding queries -> 0
               de[e] = pe[e] * (dp[8 * cc + e] - dv[e]);
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              wp[e] = pack_bf16(pe[2 * e], pe[2 * e + 1]);
-              ws[e] = pack_bf16(de[2 * e], de[2 * e + 1]);
+              wp[jj][4 * cc + e] = pack_bf16(pe[2 * e], pe[2 * e + 1]);
+              ws[jj][4 * cc + e] = pack_bf16(de[2 * e], de[2 * e + 1]);
             }
           } else {
-            wp[0] = wp[1] = wp[2] = wp[3] = 0u;
-            ws[0] = ws[1] = ws[2] = ws[3] = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) wp[jj][4 * cc + e] = ws[jj][4 * cc + e] = 0u;
           }
-          const int ch = ((4 * jj + cc) ^ (r & 7)) << 4;
-          *reinterpret_cast<uint4*>(prow + ch) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
-          *reinterpret_cast<uint4*>(srow + ch) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
         }
       }
+      // the previous chunk's dV/dK/dQ products must be done reading the P/dS tiles
+      if (!all_ok(mbar_wait(bar + 8 * C::bPDSFree, (G & 1) ^ 1))) return kErrPDSFree;
+      uint8_t* prow = gbase + C::oP + hf * kSlab + r * 128;
+      uint8_t* srow = gbase + C::oDS + hf * kSlab + r * 128;
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int ch = ((4 * jj + cc) ^ (r & 7)) << 4;
+          *reinterpret_cast<uint4*>(prow + ch) = make_uint4(
+              wp[jj][4 * cc], wp[jj][4 * cc + 1], wp[jj][4 * cc + 2], wp[jj][4 * cc + 3]);
+          *reinterpret_cast<uint4*>(srow + ch) = make_uint4(
+              ws[jj][4 * cc], ws[jj][4 * cc + 1], ws[jj][4 * cc + 2], ws[jj][4 * cc + 3]);
+        }
       fence_proxy_async_smem();
       mbar_arrive(bar + 8 * C::bPDSFull);
     }
@@ -346,8 +384,9 @@ __device__ int dq_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32_t
       tc_fence_before();
       mbar_arrive(bar + 8 * C::bDQFree);
       fence_proxy_async_smem();
-      named_barrier(1, 128);
+      mbar_arrive(bar + 8 * C::bStg);  // this thread's row of the staged dQ_c is written
       if (leader) {
+        if (!mbar_wait(bar + 8 * C::bStg, G & 1)) return kErrStg;
         const uint32_t sstg = base + C::oQ + st * 2 * C::kTile;
         const int q0 = (x.I0 + 4 * c) * kBlock;
 #pragma unroll
@@ -376,8 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar + 8 * C::bKVFull, 1);
-    mbar_init(bar + 8 * C::bKVFree, 1);
+    for (int i = 0; i < C::NKV; ++i) {
+      mbar_init(bar + 8 * (C::bKVFull + i), 1);
+      mbar_init(bar + 8 * (C::bKVFree + i), 1);
+    }
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(bar + 8 * (C::bQDFull + i), 1);
       mbar_init(bar + 8 * (C::bQDFree + i), 1);
@@ -390,6 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDQFree, 128);
     mbar_init(bar + 8 * C::bDKVFull, 1);
     mbar_init(bar + 8 * C::bDKVFree, 256);
+    mbar_init(bar + 8 * C::bStg, 128);
     mbar_init(bar + 8 * C::bDone, 1);
     fence_barrier_init();
   }

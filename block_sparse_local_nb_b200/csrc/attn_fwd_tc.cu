@@ -10,7 +10,7 @@
 // walks the items; consecutive CTAs take neighbouring tiles at the same time,
 // so the key/value blocks their windows share are served from L2.
 //
-// Warp roles (256 threads):
+// Warp roles (320 threads):
 //   warp 0     TMA producer: Q tile, then K and V chunks, into 128-byte
 //              swizzled shared memory (3-D tensor maps; rows outside [0, n)
 //              are zero-filled by TMA and masked).
@@ -19,15 +19,18 @@
 //                O  += P_c V_c   (M 128, N d,   K 128) -> TMEM, two buffers
 //              S_{c+1} is issued before P_c V_c so the softmax of the next
 //              chunk overlaps the P V product.
-//   warps 4-7  softmax: thread r owns row r (TMEM lane r).  Per chunk it reads
-//              its 128 scores, masks keys outside its query block's band or
-//              past the length, updates the running max and sum (base 2), and
-//              writes P = 2^(s - m) as bf16 into shared memory for the P V
-//              product.  The running output lives in TMEM; it is rescaled
-//              (load, multiply, store) only when the row max grows by more
-//              than 2^8, otherwise the stale max is kept (P <= 2^8, exact after
-//              the final division).  Epilogue: O / l -> bf16, lse = m + log l.
-//   warps 2-3  idle.
+//   warps 2-9  softmax, two groups of four warps; thread (r, half) owns row r
+//              (TMEM lane r) and 64 of the chunk's 128 key columns.  Per chunk
+//              it reads its 64 scores, masks keys outside its query block's
+//              band or past the length, exchanges the partial row max with the
+//              other half through shared memory, updates the running max and
+//              sum (base 2) and writes P = 2^(s - m) as bf16 into its half of
+//              the shared-memory P tile.  The running output lives in TMEM; it
+//              is rescaled (load, multiply, store; each half its own columns)
+//              only when the row max grows by more than 2^8, otherwise the
+//              stale max is kept (P <= 2^8, exact after the final division).
+//              Epilogue (deferred past the next item's first chunk): the two
+//              partial sums are combined, O / l -> bf16, lse = m + log l.
 // Every mbarrier wait is bounded; on a timeout the kernel records an error
 // code in the caller-visible error word and tears down (frees TMEM) instead
 // of hanging.
@@ -42,7 +45,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 320;
 constexpr int kRows = 128;   // query rows per tile
 constexpr int kChunk = 128;  // keys per chunk
 constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 64 bf16
@@ -54,7 +57,7 @@ template <int D>
 struct Cfg {
   static constexpr int NQ = D == 64 ? 2 : 1;   // Q tile buffers
   static constexpr int NKV = D == 64 ? 3 : 2;  // K/V chunk stages
-  static constexpr int NP = 2;                 // P buffers
+  static constexpr int NP = D == 64 ? 2 : 1;   // P buffers
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kKBytes = kChunk * D * 2;
   static constexpr int kPBytes = kRows * kChunk * 2;
@@ -67,9 +70,13 @@ struct Cfg {
   static constexpr int bQFull = 0, bQFree = bQFull + NQ, bKVFull = bQFree + NQ,
                        bKVFree = bKVFull + NKV, bSFull = bKVFree + NKV, bSFree = bSFull + 2,
                        bPFull = bSFree + 2, bPFree = bPFull + NP, bOFull = bPFree + NP,
-                       bOFree = bOFull + 2, bDone = bOFree + 2, nBar = bDone + 1;
+                       bOFree = bOFull + 2, bXMax = bOFree + 2, bXSum = bXMax + 2,
+                       bDone = bXSum + 2, nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
-  static constexpr int kSmem = oSlot + 16 + 1024;  // + slack for 1024-byte alignment
+  // exchange buffers of the two softmax halves: [parity][half][row] fp32
+  static constexpr int oXMax = oSlot + 16;
+  static constexpr int oXSum = oXMax + 2 * 2 * 128 * 4;
+  static constexpr int kSmem = oXSum + 2 * 2 * 128 * 4 + 1024;  // + slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t tS = 0;    // S buffers: columns [0,128) and [128,256)
   static constexpr uint32_t tO = 256;  // O buffers: [256, 256+D) and [256+D, 256+2D)
@@ -108,7 +115,7 @@ __device__ __forceinline__ Item decode(const Params& p, int it) {
 
 // error codes: 0x10 + site
 enum : int { kErrQFree = 0x11, kErrKVFree, kErrQFull, kErrKVFull, kErrSFree, kErrOFree, kErrPFull,
-             kErrSFull, kErrPFree, kErrPPrev, kErrOFull, kErrDone };
+             kErrSFull, kErrPFree, kErrPPrev, kErrOFull, kErrDone, kErrXMax, kErrXSum };
 
 template <int D>
 __device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tq,
@@ -151,14 +158,40 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
   const uint32_t bar = base + C::oBar;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, kChunk, false, false);  // Q K^T: both K-major
   constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);       // P V: V is MN-major
-  int g = 0, tc = 0;
+  // S of chunk G+1 is issued before P V of chunk G, also across items, so the
+  // softmax of the next chunk never waits behind a P V product.
+  struct Pending {
+    bool valid;
+    int G, c, tc;
+    bool last;
+  } pend = {false, 0, 0, 0, false};
+  auto issue_pv = [&](const Pending& q) -> int {
+    const int st = q.G % C::NKV, pb = q.G % C::NP, ob = q.tc % 2;
+    if (q.c == 0 && !mbar_wait(bar + 8 * (C::bOFree + ob), ((q.tc / 2) & 1) ^ 1)) return kErrOFree;
+    if (!mbar_wait(bar + 8 * (C::bPFull + pb), (q.G / C::NP) & 1)) return kErrPFull;
+    tc_fence_after();
+    const uint32_t sP = base + C::oP + pb * C::kPBytes;
+    const uint32_t sV = base + C::oV + st * C::kKBytes;
+#pragma unroll
+    for (int k = 0; k < kChunk / 16; ++k) {
+      const uint64_t ad = smem_desc_sw128(sP + (k >> 2) * kSlab + (k & 3) * 32, 0, 1024);
+      // V is MN-major: 64-column swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
+      mma_bf16_ss(tmem + C::tO + ob * D, ad, smem_desc_sw128(sV + k * 2048, kSlab, 1024), kIdPV,
+                  q.c > 0 || k > 0);
+    }
+    mma_commit(bar + 8 * (C::bKVFree + st));
+    mma_commit(bar + 8 * (C::bPFree + pb));
+    if (q.last) mma_commit(bar + 8 * (C::bOFull + ob));
+    return 0;
+  };
+  int g = 0, tc = 0, e = 0;
   for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
     const Item x = decode(p, it);
     if (x.nch == 0) continue;
-    const int qs = tc % C::NQ, ob = tc % 2;
+    const int qs = tc % C::NQ;
     if (!mbar_wait(bar + 8 * (C::bQFull + qs), (tc / C::NQ) & 1)) return kErrQFull;
     const uint32_t sQ = base + C::oQ + qs * C::kQBytes;
-    auto issue_s = [&](int c) -> int {
+    for (int c = 0; c < x.nch; ++c) {
       const int G = g + c, st = G % C::NKV, sb = G % 2;
       if (!mbar_wait(bar + 8 * (C::bKVFull + st), (G / C::NKV) & 1)) return kErrKVFull;
       if (!mbar_wait(bar + 8 * (C::bSFree + sb), ((G / 2) & 1) ^ 1)) return kErrSFree;
@@ -171,42 +204,20 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
                     smem_desc_sw128(sK + off, 0, 1024), kIdS, k > 0);
       }
       mma_commit(bar + 8 * (C::bSFull + sb));
-      return 0;
-    };
-    int e = issue_s(0);
-    if (e) return e;
-    for (int c = 0; c < x.nch; ++c) {
-      if (c + 1 < x.nch) {
-        if ((e = issue_s(c + 1))) return e;
-      } else {
-        mma_commit(bar + 8 * (C::bQFree + qs));  // all S products of this tile issued
-      }
-      const int G = g + c, st = G % C::NKV, pb = G % C::NP;
-      if (c == 0 && !mbar_wait(bar + 8 * (C::bOFree + ob), ((tc / 2) & 1) ^ 1)) return kErrOFree;
-      if (!mbar_wait(bar + 8 * (C::bPFull + pb), (G / C::NP) & 1)) return kErrPFull;
-      tc_fence_after();
-      const uint32_t sP = base + C::oP + pb * C::kPBytes;
-      const uint32_t sV = base + C::oV + st * C::kKBytes;
-#pragma unroll
-      for (int k = 0; k < kChunk / 16; ++k) {
-        const uint64_t ad = smem_desc_sw128(sP + (k >> 2) * kSlab + (k & 3) * 32, 0, 1024);
-        // V is MN-major: 64-column swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
-        mma_bf16_ss(tmem + C::tO + ob * D, ad, smem_desc_sw128(sV + k * 2048, kSlab, 1024), kIdPV,
-                    c > 0 || k > 0);
-      }
-      mma_commit(bar + 8 * (C::bKVFree + st));
-      mma_commit(bar + 8 * (C::bPFree + pb));
-      if (c == x.nch - 1) mma_commit(bar + 8 * (C::bOFull + ob));
+      if (c == x.nch - 1) mma_commit(bar + 8 * (C::bQFree + qs));  // the tile's S products issued
+      if (pend.valid && (e = issue_pv(pend))) return e;
+      pend = {true, G, c, tc, c == x.nch - 1};
     }
     g += x.nch;
     ++tc;
   }
+  if (pend.valid && (e = issue_pv(pend))) return e;
   return 0;
 }
 
 template <int D>
 __device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, uint32_t tmem,
-                                int wq, int lane) {
+                                int wq, int hf, int lane) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
@@ -214,18 +225,67 @@ __device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, 
   const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   const int nb = a.n / kBlock;
   const float sl2 = a.scale * kLog2e;
+  float* xmax = reinterpret_cast<float*>(gbase + C::oXMax);
+  float* xsum = reinterpret_cast<float*>(gbase + C::oXSum);
   auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
-  int g = 0, tc = 0;
+  // An item's epilogue runs after the next item's first chunk, so the wait for
+  // its last P V product overlaps that chunk's softmax.
+  struct Epi {
+    bool valid;
+    int tc;
+    int64_t row;  // global row index of this thread's query (bh * n + q)
+    bool in_range, row_valid;
+    float m, l;   // running max (base 2) and this half's partial sum
+  } pend = {false, 0, 0, false, false, 0.f, 0.f};
+  auto epilogue = [&](const Epi& x) -> int {
+    const int ob = x.tc % 2, par = x.tc & 1;
+    xsum[(par * 2 + hf) * 128 + r] = x.l;
+    mbar_arrive(bar + 8 * (C::bXSum + par));
+    if (!all_ok(mbar_wait(bar + 8 * (C::bXSum + par), (x.tc >> 1) & 1))) return kErrXSum;
+    const float l = x.l + xsum[(par * 2 + (hf ^ 1)) * 128 + r];
+    if (!all_ok(mbar_wait(bar + 8 * (C::bOFull + ob), (x.tc / 2) & 1))) return kErrOFull;
+    tc_fence_after();
+    float o[D / 64][32];
+#pragma unroll
+    for (int j = 0; j < D / 64; ++j) tmem_ld32(trow + C::tO + ob * D + hf * (D / 2) + 32 * j, o[j]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < D / 64; ++j) reg_fence(o[j]);
+    tc_fence_before();
+    mbar_arrive(bar + 8 * (C::bOFree + ob));
+    const bool has = x.row_valid && l > 0.f;
+    const float inv = has ? 1.f / l : 0.f;
+    if (x.in_range) {
+      uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) +
+                                             x.row * D + hf * (D / 2));
+#pragma unroll
+      for (int j = 0; j < D / 64; ++j) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 u;
+          u.x = pack_bf16(o[j][8 * v + 0] * inv, o[j][8 * v + 1] * inv);
+          u.y = pack_bf16(o[j][8 * v + 2] * inv, o[j][8 * v + 3] * inv);
+          u.z = pack_bf16(o[j][8 * v + 4] * inv, o[j][8 * v + 5] * inv);
+          u.w = pack_bf16(o[j][8 * v + 6] * inv, o[j][8 * v + 7] * inv);
+          orow[4 * j + v] = u;
+        }
+      }
+      if (a.lse && hf == 0) a.lse[x.row] = has ? (x.m + log2f(l)) * kLn2 : -INFINITY;
+    }
+    return 0;
+  };
+  int g = 0, tc = 0, e = 0;
   for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
     const Item x = decode(p, it);
     const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
     const int q = x.tile * kRows + r;
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) + (bh * a.n + q) * D;
     if (x.nch == 0) {  // the whole tile is padding
       if (q < a.n) {
+        uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) +
+                                               (bh * a.n + q) * D + hf * (D / 2));
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) reinterpret_cast<uint4*>(orow)[i] = make_uint4(0, 0, 0, 0);
-        if (a.lse) a.lse[bh * a.n + q] = -INFINITY;
+        for (int i = 0; i < D / 16; ++i) orow[i] = make_uint4(0, 0, 0, 0);
+        if (a.lse && hf == 0) a.lse[bh * a.n + q] = -INFINITY;
       }
       continue;
     }
@@ -233,42 +293,70 @@ __device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, 
     const bool row_valid = q < x.L;
     float m_used = -INFINITY, l = 0.f;
     for (int c = 0; c < x.nch; ++c) {
-      const int G = g + c, sb = G % 2, pb = G % C::NP;
+      const int G = g + c, sb = G % 2, pb = G % C::NP, par = G & 1;
       if (!all_ok(mbar_wait(bar + 8 * (C::bSFull + sb), (G / 2) & 1))) return kErrSFull;
       tc_fence_after();
-      float s[4][32];
+      float s[2][32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) tmem_ld32(trow + C::tS + sb * kChunk + 32 * j, s[j]);
+      for (int j = 0; j < 2; ++j) tmem_ld32(trow + C::tS + sb * kChunk + 64 * hf + 32 * j, s[j]);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 4; ++j) reg_fence(s[j]);
+      for (int j = 0; j < 2; ++j) reg_fence(s[j]);
       tc_fence_before();
       mbar_arrive(bar + 8 * (C::bSFree + sb));
 
-      bool vis[4];
-      float cmax = -INFINITY;
+      bool vis[2];
+      float pm[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int kb = x.J0 + 4 * c + j;
+      for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int kb = x.J0 + 4 * c + 2 * hf + j;
         vis[j] = row_valid && kb < nb && abs(kb - qb) <= a.R && kb * kBlock < x.L;
         if (vis[j]) {
           const int lim = x.L - kb * kBlock;  // keys at or past the length are masked
+          if (lim < 32) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float v = i < lim ? s[j][i] * sl2 : -INFINITY;
-            s[j][i] = v;
-            cmax = fmaxf(cmax, v);
+            for (int i = 0; i < 32; ++i) s[j][i] = i < lim ? s[j][i] : -INFINITY;
           }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[j][i]);
         }
       }
+      float cmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                         fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      // combine with the other half's partial max (raw units; the scale is positive)
+      xmax[(par * 2 + hf) * 128 + r] = cmax;
+      mbar_arrive(bar + 8 * (C::bXMax + par));
+      if (!all_ok(mbar_wait(bar + 8 * (C::bXMax + par), (G >> 1) & 1))) return kErrXMax;
+      cmax = fmaxf(cmax, xmax[(par * 2 + (hf ^ 1)) * 128 + r]) * sl2;
       bool need = false;
       float alpha = 1.f;
       if (cmax > m_used + kTau) {
         if (m_used != -INFINITY) {
           need = true;
-          alpha = exp2f(m_used - cmax);
+          alpha = ex2_approx(m_used - cmax);
         }
         m_used = cmax;
+      }
+      // P = 2^(s scale log2e - m) in bf16 for this half's 64 keys
+      const float nm = -m_used;
+      uint32_t w[2][16];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        if (vis[j]) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2_approx(fmaf(s[j][2 * i], sl2, nm));
+            const float p1 = ex2_approx(fmaf(s[j][2 * i + 1], sl2, nm));
+            ls[i & 3] += p0 + p1;
+            w[j][i] = pack_bf16(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[j][i] = 0u;
+        }
       }
       if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + pb), ((G / C::NP) & 1) ^ 1))) return kErrPFree;
       if (__any_sync(0xffffffffu, need)) {
@@ -277,9 +365,9 @@ __device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, 
         if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + Gp % C::NP), (Gp / C::NP) & 1)))
           return kErrPPrev;
         tc_fence_after();
-        const uint32_t to = trow + C::tO + (tc % 2) * D;
+        const uint32_t to = trow + C::tO + (tc % 2) * D + hf * (D / 2);
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
+        for (int j = 0; j < D / 64; ++j) {
           float ov[32];
           tmem_ld32(to + 32 * j, ov);
           tmem_wait_ld();
@@ -291,66 +379,28 @@ __device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, 
         tmem_wait_st();
         l *= alpha;
       }
-      // P = 2^(s - m) in bf16, row r of the 128-byte-swizzled P tile
-      uint8_t* prow = gbase + C::oP + pb * C::kPBytes + r * 128;
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      // this half's 64 keys are exactly slab hf of the 128-byte-swizzled P tile
+      uint8_t* prow = gbase + C::oP + pb * C::kPBytes + hf * kSlab + r * 128;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int chunk = 4 * j + cc;  // 8 keys per 16-byte chunk
-          uint32_t w[4];
-          if (vis[j]) {
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-              const float p0 = exp2f(s[j][8 * cc + 2 * e2] - m_used);
-              const float p1 = exp2f(s[j][8 * cc + 2 * e2 + 1] - m_used);
-              l += p0 + p1;
-              w[e2] = pack_bf16(p0, p1);
-            }
-          } else {
-            w[0] = w[1] = w[2] = w[3] = 0u;
-          }
-          const int slab = chunk >> 3, c8 = chunk & 7;
-          *reinterpret_cast<uint4*>(prow + slab * kSlab + ((c8 ^ (r & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-        }
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const int j = c8 >> 2, i0 = (c8 & 3) * 4;
+        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) =
+            make_uint4(w[j][i0], w[j][i0 + 1], w[j][i0 + 2], w[j][i0 + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar + 8 * (C::bPFull + pb));
-    }
-    // epilogue: O / l
-    const int ob = tc % 2;
-    if (!all_ok(mbar_wait(bar + 8 * (C::bOFull + ob), (tc / 2) & 1))) return kErrOFull;
-    tc_fence_after();
-    float o[D / 32][32];
-#pragma unroll
-    for (int j = 0; j < D / 32; ++j) tmem_ld32(trow + C::tO + ob * D + 32 * j, o[j]);
-    tmem_wait_ld();
-#pragma unroll
-    for (int j = 0; j < D / 32; ++j) reg_fence(o[j]);
-    tc_fence_before();
-    mbar_arrive(bar + 8 * (C::bOFree + ob));
-    const bool has = row_valid && l > 0.f;
-    const float inv = has ? 1.f / l : 0.f;
-    if (q < a.n) {
-#pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 u;
-          u.x = pack_bf16(o[j][8 * v + 0] * inv, o[j][8 * v + 1] * inv);
-          u.y = pack_bf16(o[j][8 * v + 2] * inv, o[j][8 * v + 3] * inv);
-          u.z = pack_bf16(o[j][8 * v + 4] * inv, o[j][8 * v + 5] * inv);
-          u.w = pack_bf16(o[j][8 * v + 6] * inv, o[j][8 * v + 7] * inv);
-          reinterpret_cast<uint4*>(orow)[4 * j + v] = u;
-        }
+      if (c == 0 && pend.valid) {  // the previous item's epilogue, deferred past this chunk
+        if ((e = epilogue(pend))) return e;
+        pend.valid = false;
       }
-      if (a.lse) a.lse[bh * a.n + q] = has ? (m_used + log2f(l)) * kLn2 : -INFINITY;
     }
+    pend = {true, tc, bh * a.n + q, q < a.n, row_valid, m_used, l};
     g += x.nch;
     ++tc;
   }
+  if (pend.valid && (e = epilogue(pend))) return e;
   return 0;
 }
 
@@ -377,12 +427,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + 8 * (C::bSFull + i), 1);
-      mbar_init(bar + 8 * (C::bSFree + i), 128);
+      mbar_init(bar + 8 * (C::bSFree + i), 256);
       mbar_init(bar + 8 * (C::bOFull + i), 1);
-      mbar_init(bar + 8 * (C::bOFree + i), 128);
+      mbar_init(bar + 8 * (C::bOFree + i), 256);
+      mbar_init(bar + 8 * (C::bXMax + i), 256);
+      mbar_init(bar + 8 * (C::bXSum + i), 256);
     }
     for (int i = 0; i < C::NP; ++i) {
-      mbar_init(bar + 8 * (C::bPFull + i), 128);
+      mbar_init(bar + 8 * (C::bPFull + i), 256);
       mbar_init(bar + 8 * (C::bPFree + i), 1);
     }
     mbar_init(bar + 8 * C::bDone, 1);
@@ -407,8 +459,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) err = producer<D>(p, base, &tq, &tk, &tv);
   } else if (warp == 1) {
     if (lane == 0) err = mma_issuer<D>(p, base, tmem);
-  } else if (warp >= 4) {
-    err = softmax_epilogue<D>(p, base, gbase, tmem, warp - 4, lane);
+  } else {
+    err = softmax_epilogue<D>(p, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane);
   }
   if (err) record_error(p.a.err, err);
 

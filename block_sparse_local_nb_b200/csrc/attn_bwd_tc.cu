@@ -40,30 +40,37 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
-  // D = 64: K/V tiles double-buffered and S/dP of chunk G+1 issued before the
-  // dV/dK/dQ products of chunk G (the gradient warps of G+1 then overlap them).
-  // D = 128: TMEM is full (dQ reuses the S columns), so chunks run in order.
+  // D = 64: K/V tiles double-buffered; S/dP of chunk G+1 issued before the
+  // dV/dK/dQ products of chunk G (the gradient warps of G+1 then overlap them);
+  // P^T kept in TMEM (64 spare columns) as the A operand of dV, which leaves
+  // room for a dQ staging buffer of its own.
+  // D = 128: TMEM is full (dQ reuses the S columns), so chunks run in order,
+  // P^T goes through shared memory and dQ is staged in the chunk's Q/dO buffer.
   static constexpr bool kLook = D == 64;
+  static constexpr bool kPTmem = D == 64;
   static constexpr int NKV = D == 64 ? 2 : 1;  // K/V tile buffers
-  static constexpr int NS = D == 64 ? 2 : 1;   // Q/dO chunk stages
+  static constexpr int NS = D == 64 ? 3 : 1;   // Q/dO chunk stages
   static constexpr int kTile = kRows * D * 2;  // one [128 x D] bf16 tile
   static constexpr int kPT = kRows * kRows * 2;  // one [128 x 128] bf16 tile
   static constexpr int oK = 0;                   // buffer i: K at oK + 2 i kTile, V after it
   static constexpr int oQ = NKV * 2 * kTile;     // stage s: Q at oQ + 2 s kTile, dO after it
-  static constexpr int oP = oQ + NS * 2 * kTile;
-  static constexpr int oDS = oP + kPT;
-  static constexpr int oLD = oDS + kPT;  // stage s: -lse log2e [128] then D [128], fp32
+  static constexpr int oP = oQ + NS * 2 * kTile;  // P^T tile (shared-memory variant only)
+  static constexpr int oDS = oP + (kPTmem ? 0 : kPT);
+  static constexpr int oStg = oDS + kPT;  // dQ staging box (TMEM-P variant only)
+  static constexpr int oLD = oStg + (kPTmem ? kSlab : 0);  // stage s: -lse log2e, D
   static constexpr int oBar = oLD + NS * 1024;
   static constexpr int bKVFull = 0, bKVFree = bKVFull + NKV, bQDFull = bKVFree + NKV,
                        bQDFree = bQDFull + NS, bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1,
                        bPDSFull = bSDPFree + 1, bPDSFree = bPDSFull + 1, bDQFull = bPDSFree + 1,
                        bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
-                       bStg = bDKVFree + 1, bDone = bStg + 1, nBar = bDone + 1;
+                       bStg = bDKVFree + 1, bStgFree = bStg + 1, bDone = bStgFree + 1,
+                       nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
   static constexpr int kSmem = oSlot + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D;
   static constexpr uint32_t tDQ = D == 64 ? 384 : 0;  // for D = 128, dQ reuses the S columns
+  static constexpr uint32_t tP = 448;                 // P^T, bf16 pairs (TMEM-P variant)
 };
 
 struct Params {
@@ -100,7 +107,7 @@ __device__ __forceinline__ Item decode(const Params& p, int it) {
 
 enum : int { kErrKVFree = 0x31, kErrQDFree, kErrKVFull, kErrQDFull, kErrSDPFree, kErrDQFree,
              kErrPDSFull, kErrDKVFree, kErrGQD, kErrSDPFull, kErrPDSFree, kErrDKVFull,
-             kErrDQFull, kErrDone, kErrStg };
+             kErrDQFull, kErrDone, kErrStg, kErrStgFree };
 
 template <int D>
 __device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tk,
@@ -171,8 +178,12 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
 #pragma unroll
     for (int k = 0; k < kRows / 16; ++k) {  // k over the chunk's queries
       const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
-      mma_bf16_ss(tmem + C::tDV, smem_desc_sw128(sP + off, 0, 1024),
-                  smem_desc_sw128(sdO + k * 2048, kSlab, 1024), kIdKV, q.c > 0 || k > 0);
+      if (C::kPTmem)
+        mma_bf16_ts(tmem + C::tDV, tmem + C::tP + 8 * k,
+                    smem_desc_sw128(sdO + k * 2048, kSlab, 1024), kIdKV, q.c > 0 || k > 0);
+      else
+        mma_bf16_ss(tmem + C::tDV, smem_desc_sw128(sP + off, 0, 1024),
+                    smem_desc_sw128(sdO + k * 2048, kSlab, 1024), kIdKV, q.c > 0 || k > 0);
       mma_bf16_ss(tmem + C::tDK, smem_desc_sw128(sS + off, 0, 1024),
                   smem_desc_sw128(sQ + k * 2048, kSlab, 1024), kIdKV, q.c > 0 || k > 0);
     }
@@ -182,6 +193,7 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
                   smem_desc_sw128(sK + k * 2048, kSlab, 1024), kIdQ, k > 0);
     mma_commit(bar + 8 * C::bPDSFree);
     mma_commit(bar + 8 * C::bDQFull);
+    if (C::kPTmem) mma_commit(bar + 8 * (C::bQDFree + q.st));  // Q/dO of the chunk consumed
     if (q.last) {
       mma_commit(bar + 8 * C::bDKVFull);
       mma_commit(bar + 8 * (C::bKVFree + q.kvb));
@@ -260,7 +272,7 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
       tc_fence_after();
       const float* nl = reinterpret_cast<const float*>(gbase + C::oLD + st * 1024);
       const float* Dv = nl + 128;
-      uint32_t wp[2][16], ws[2][16];  // packed bf16 P^T and dS^T for this thread's 64 queries
+      uint32_t wp[32], ws[32];  // packed bf16 P^T and dS^T for this thread's 64 queries
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
         const int j = 2 * hf + jj;  // 32-query group within the chunk
@@ -293,12 +305,12 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              wp[jj][4 * cc + e] = pack_bf16(pe[2 * e], pe[2 * e + 1]);
-              ws[jj][4 * cc + e] = pack_bf16(de[2 * e], de[2 * e + 1]);
+              wp[16 * jj + 4 * cc + e] = pack_bf16(pe[2 * e], pe[2 * e + 1]);
+              ws[16 * jj + 4 * cc + e] = pack_bf16(de[2 * e], de[2 * e + 1]);
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) wp[jj][4 * cc + e] = ws[jj][4 * cc + e] = 0u;
+            for (int e = 0; e < 4; ++e) wp[16 * jj + 4 * cc + e] = ws[16 * jj + 4 * cc + e] = 0u;
           }
         }
       }
@@ -306,17 +318,25 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
       if (!all_ok(mbar_wait(bar + 8 * C::bPDSFree, (G & 1) ^ 1))) return kErrPDSFree;
       uint8_t* prow = gbase + C::oP + hf * kSlab + r * 128;
       uint8_t* srow = gbase + C::oDS + hf * kSlab + r * 128;
+      if (C::kPTmem) {  // this thread's 64 queries = 32 packed columns of P^T in TMEM
+        tmem_st32u(trow + C::tP + 32 * hf, wp);
+      }
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           const int ch = ((4 * jj + cc) ^ (r & 7)) << 4;
-          *reinterpret_cast<uint4*>(prow + ch) = make_uint4(
-              wp[jj][4 * cc], wp[jj][4 * cc + 1], wp[jj][4 * cc + 2], wp[jj][4 * cc + 3]);
-          *reinterpret_cast<uint4*>(srow + ch) = make_uint4(
-              ws[jj][4 * cc], ws[jj][4 * cc + 1], ws[jj][4 * cc + 2], ws[jj][4 * cc + 3]);
+          if (!C::kPTmem)
+            *reinterpret_cast<uint4*>(prow + ch) =
+                make_uint4(wp[16 * jj + 4 * cc], wp[16 * jj + 4 * cc + 1],
+                           wp[16 * jj + 4 * cc + 2], wp[16 * jj + 4 * cc + 3]);
+          *reinterpret_cast<uint4*>(srow + ch) =
+              make_uint4(ws[16 * jj + 4 * cc], ws[16 * jj + 4 * cc + 1], ws[16 * jj + 4 * cc + 2],
+                         ws[16 * jj + 4 * cc + 3]);
         }
+      if (C::kPTmem) tmem_wait_st();
       fence_proxy_async_smem();
+      tc_fence_before();
       mbar_arrive(bar + 8 * C::bPDSFull);
     }
     // epilogue: first group writes dK (times 1/sqrt(d)), second group dV
@@ -366,34 +386,66 @@ __device__ int dq_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32_t
     const int bh = x.b * a.heads + x.h;
     for (int c = 0; c < x.nch; ++c) {
       const int G = g + c, st = G % C::NS;
+      const int q0 = (x.I0 + 4 * c) * kBlock;
       if (!all_ok(mbar_wait(bar + 8 * C::bDQFull, G & 1))) return kErrDQFull;
       tc_fence_after();
-      // stage dQ_c (fp32) in the chunk's Q/dO buffer, laid out as D/32 swizzled boxes
-      uint8_t* stg = gbase + C::oQ + st * 2 * C::kTile;
+      if constexpr (C::kPTmem) {
+        // whole dQ_c row in registers, then one 32-column box per pass through the
+        // staging buffer
+        float v[D / 32][32];
 #pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-        float v[32];
-        tmem_ld32(trow + C::tDQ + 32 * j, v);
+        for (int j = 0; j < D / 32; ++j) tmem_ld32(trow + C::tDQ + 32 * j, v[j]);
         tmem_wait_ld();
-        reg_fence(v);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<float4*>(stg + j * kSlab + r * 128 + ((u ^ (r & 7)) << 4)) =
-              make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-      }
-      tc_fence_before();
-      mbar_arrive(bar + 8 * C::bDQFree);
-      fence_proxy_async_smem();
-      mbar_arrive(bar + 8 * C::bStg);  // this thread's row of the staged dQ_c is written
-      if (leader) {
-        if (!mbar_wait(bar + 8 * C::bStg, G & 1)) return kErrStg;
-        const uint32_t sstg = base + C::oQ + st * 2 * C::kTile;
-        const int q0 = (x.I0 + 4 * c) * kBlock;
+        for (int j = 0; j < D / 32; ++j) reg_fence(v[j]);
+        tc_fence_before();
+        mbar_arrive(bar + 8 * C::bDQFree);
+        uint8_t* stg = gbase + C::oStg;
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) tma_reduce_add_3d(tdq, sstg + j * kSlab, 32 * j, q0, bh);
-        bulk_commit();
-        bulk_wait_read0();
-        mbar_arrive(bar + 8 * (C::bQDFree + st));
+        for (int j = 0; j < D / 32; ++j) {
+          const int k = G * (D / 32) + j;  // global pass index
+          if (!all_ok(mbar_wait(bar + 8 * C::bStgFree, (k & 1) ^ 1))) return kErrStgFree;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4*>(stg + r * 128 + ((u ^ (r & 7)) << 4)) =
+                make_float4(v[j][4 * u], v[j][4 * u + 1], v[j][4 * u + 2], v[j][4 * u + 3]);
+          fence_proxy_async_smem();
+          mbar_arrive(bar + 8 * C::bStg);  // this thread's row of the box is written
+          if (leader) {
+            if (!mbar_wait(bar + 8 * C::bStg, k & 1)) return kErrStg;
+            tma_reduce_add_3d(tdq, base + C::oStg, 32 * j, q0, bh);
+            bulk_commit();
+            bulk_wait_read0();
+            mbar_arrive(bar + 8 * C::bStgFree);
+          }
+        }
+      } else {
+        // all D/32 boxes at once in the chunk's Q/dO buffer (free once dQ_c is done)
+        uint8_t* stg = gbase + C::oQ + st * 2 * C::kTile;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          float v[32];
+          tmem_ld32(trow + C::tDQ + 32 * j, v);
+          tmem_wait_ld();
+          reg_fence(v);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4*>(stg + j * kSlab + r * 128 + ((u ^ (r & 7)) << 4)) =
+                make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        }
+        tc_fence_before();
+        mbar_arrive(bar + 8 * C::bDQFree);
+        fence_proxy_async_smem();
+        mbar_arrive(bar + 8 * C::bStg);
+        if (leader) {
+          if (!mbar_wait(bar + 8 * C::bStg, G & 1)) return kErrStg;
+#pragma unroll
+          for (int j = 0; j < D / 32; ++j)
+            tma_reduce_add_3d(tdq, base + C::oQ + st * 2 * C::kTile + j * kSlab, 32 * j, q0, bh);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(bar + 8 * (C::bQDFree + st));
+        }
       }
     }
     g += x.nch;
@@ -432,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDKVFull, 1);
     mbar_init(bar + 8 * C::bDKVFree, 256);
     mbar_init(bar + 8 * C::bStg, 128);
+    mbar_init(bar + 8 * C::bStgFree, 1);
     mbar_init(bar + 8 * C::bDone, 1);
     fence_barrier_init();
   }

@@ -259,6 +259,67 @@ def cpu_baseline(w):
                       f"host has {os.cpu_count()} logical cores"}
 
 
+def run_tokenizer_workload(args):
+    """The 2**28-byte k-mer tokenizer workload alone (one GPU): bases/s and the
+    fraction of the HBM roofline (1 byte read + 2.25 bytes written per base)."""
+    import torch
+
+    import block_sparse_local_nb_b200 as nb
+    from block_sparse_local_nb_b200.inputs import DNA_BYTES, make_dna
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dna = make_dna(DNA_BYTES)
+    seq = torch.from_numpy(dna).to(dev)
+    ids = torch.empty(DNA_BYTES - 5, dtype=torch.int16, device=dev)
+    packed = torch.empty(DNA_BYTES // 4, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sptr = stream.cuda_stream
+    for _ in range(args.warmup):
+        nb.nb_tokenize_kmer(seq, DNA_BYTES, ids, packed, 6, sptr)
+    torch.cuda.synchronize(dev)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(0)
+    with sampler:
+        start.record(stream)
+        for _ in range(args.steps):
+            nb.nb_tokenize_kmer(seq, DNA_BYTES, ids, packed, 6, sptr)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(end) / args.steps
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    alg_bytes = DNA_BYTES + 2 * (DNA_BYTES - 5) + DNA_BYTES // 4
+    achieved = alg_bytes / (ms / 1e3) / 1e9
+    line = {
+        "metric": "k-mer tokenizer bases/s and % of HBM roofline", "value": DNA_BYTES / (ms / 1e3),
+        "unit": "bases/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8", "data": "synthetic",
+        "config": {"workload": "dna_2p28", "bytes": DNA_BYTES, "k": 6, "n_fraction": 0.01,
+                   "l2": "inputs and outputs (872 MB) larger than the 126 MB L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": recorded_traffic("tokenize_kmer_kernel", "dna_2p28"),
+                     "kernel": "tokenize_kmer_kernel", "peak_source": peak_kind},
+        "gpu_launches": args.steps, "clocks": sampler.summary(),
+    }
+    if not args.no_cpu_baseline:
+        from threadpoolctl import threadpool_info
+
+        from oracle import kmer_ids, pack_2bit
+
+        sample = dna[: 1 << 24]
+        t0 = time.perf_counter()
+        kmer_ids(sample, 6)
+        pack_2bit(sample)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": sample.size / dt, "unit": "bases/s", "cores": 1,
+                                "kind": "oracle", "sample": "first 2**24 bytes of the workload "
+                                "through the NumPy oracle (ids + packed stream)"}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -276,6 +337,10 @@ def main():
 
     from block_sparse_local_nb_b200.inputs import WORKLOADS
 
+    if args.workload == "dna_2p28":
+        if args.impl == "native" and int(os.environ.get("RANK", "0")) == 0:
+            run_tokenizer_workload(args)
+        return
     w = WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -290,6 +355,7 @@ def main():
     import torch.distributed as dist
 
     import block_sparse_local_nb_b200 as nb
+    from block_sparse_local_nb_b200.dist import job_throughput, max_over_ranks, rank_seed
     from block_sparse_local_nb_b200.inputs import make_attn_inputs
 
     torch.cuda.set_device(local_rank)
@@ -307,7 +373,7 @@ def main():
     # ---- resident inputs: rotating sets so each step's reads miss L2
     per_set = None
     sets = []
-    base_seed = w.seed + 1000 * rank
+    base_seed = rank_seed(w.seed, rank)
     nsets = args.sets
     q0, k0, v0, do0, lengths = make_attn_inputs(w, device=dev, seed=base_seed)
     lengths_d = lengths.to(dev)
@@ -377,18 +443,14 @@ def main():
             step(sets[s % nsets], evs[s])
         end.record(stream)
         barrier()
-    elapsed_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
     tok_ms = [e[0].elapsed_time(e[1]) for e in evs]
     fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
     bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
 
     alg = algorithmic(w, lengths.tolist())
     tokens_step = alg["tokens"]
-    value = tokens_step * args.steps * world / (elapsed_ms / 1e3)
+    value = job_throughput(tokens_step, args.steps, world, elapsed_ms)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
     host = {}
@@ -419,12 +481,8 @@ def main():
             e2e_step()
         e_end.record(stream)
         barrier()
-    e2e_ms = e_start.elapsed_time(e_end)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = tokens_step * args.steps * world / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
+    e2e_value = job_throughput(tokens_step, args.steps, world, e2e_ms)
 
     if world > 1:
         dist.barrier(device_ids=[local_rank])

@@ -94,8 +94,9 @@ def test_fwd_empty_problem_is_a_no_op(lib):
 def test_bwd_workspace_size(lib):
     ws = lib.nb_attn_bwd_workspace_size(4, 12, 4096, 64, BF16)
     rows = 4 * 12 * 4096
-    assert ws >= rows * 4 + rows * 64 * 4
-    assert ws < rows * 4 + rows * 64 * 4 + 1024
+    # row term D, -lse*log2(e) and the fp32 dQ accumulator, each 256-byte aligned
+    assert ws >= 2 * rows * 4 + rows * 64 * 4
+    assert ws < 2 * rows * 4 + rows * 64 * 4 + 3 * 256
     assert lib.nb_attn_bwd_workspace_size(1, 1, 33, 64, BF16) == 0  # invalid n
     assert lib.nb_attn_bwd_workspace_size(0, 1, 64, 64, BF16) == 0
 

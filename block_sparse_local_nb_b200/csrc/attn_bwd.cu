@@ -7,7 +7,7 @@
 //     padding rows, so padding queries get P = 0 in the main kernel), and zero
 //     the fp32 dQ accumulator.
 //  2. main (attn_bwd_tc.cu): dK, dV and the dQ accumulation.
-//  3. dq_out: dQ = bf16(accumulator / sqrt(d)).
+//  3. dq_out: dQ = bf16(accumulator / sqrt(d)) on valid rows, 0 on padding rows.
 #include <math.h>
 
 #include "nb_internal.h"
@@ -49,14 +49,16 @@ __global__ void __launch_bounds__(256) bwd_rowterm_kernel(AttnArgs a, int64_t ro
         acc = fmaf(of.y, df.y, acc);
       }
     }
-    float4* z = reinterpret_cast<float4*>(w.dqacc + row * D + part * 8);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (valid) {  // padding rows of the accumulator are never read
+      float4* z = reinterpret_cast<float4*>(w.dqacc + row * D + part * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (in && part == 0) {
-    w.D[row] = acc;
+    w.D[row] = -acc;  // stored negated: the main kernel forms dP + (-D)
     w.nlse2[row] = valid ? -a.lse[row] * kLog2e : -INFINITY;
   }
 }
@@ -67,6 +69,14 @@ __global__ void __launch_bounds__(256) bwd_dq_out_kernel(AttnArgs a, int64_t row
   const int64_t nvec = rows * D / 8;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nvec;
        idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = idx / (D / 8);
+    const int64_t bh = row / a.n;
+    int L = a.lengths ? a.lengths[bh / a.heads] : a.n;
+    L = min(max(L, 0), a.n);
+    if (row - bh * a.n >= L) {  // padding row: dQ = 0, accumulator not read
+      reinterpret_cast<uint4*>(a.dq)[idx] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
     const float4 x = reinterpret_cast<const float4*>(dqacc)[2 * idx];
     const float4 y = reinterpret_cast<const float4*>(dqacc)[2 * idx + 1];
     uint4 out;

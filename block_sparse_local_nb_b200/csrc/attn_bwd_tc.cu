@@ -9,22 +9,24 @@
 // [4t - R, 4t + 3 + R], taken in chunks of 128 queries.  Per chunk, with keys
 // on the TMEM lanes (M = 128):
 //   S^T  = K Q^T          dP^T = V dO^T                       (N 128, K d)
-//   P^T  = 2^(S^T scale log2e - lse log2e),  dS^T = P^T (dP^T - D)   (CUDA cores)
+//   P^T  = 2^(S^T scale log2e - lse log2e),  dS^T = P^T (dP^T - D)   (CUDA cores,
+//          packed fp32x2 arithmetic)
 //   dV  += P^T dO         dK  += dS^T Q                        (N d, K 128)
 //   dQ_c = dS K           (queries on the lanes: dS^T read as an MN-major A)
 // dK and dV accumulate in TMEM over the item's chunks (deterministic); dQ_c is
 // added into an fp32 accumulator in global memory with a TMA bulk reduce-add.
 //
-// Warp roles (448 threads): warp 0 TMA producer (K, V tiles; Q, dO chunks;
-// the chunk's lse and D rows by bulk copy); warp 1 TMEM owner and MMA issuer;
-// warps 2-9 gradient warps: two groups of four, one per half of the chunk's
-// query columns, thread = key row; they also write dK (first group) and dV
-// (second group) at the end of an item; warps 10-13 dQ warps: thread = query
-// row, stage dQ_c in shared memory (reusing the chunk's Q/dO buffer) and
+// Warp roles (512 threads, four warpgroups with reallocated registers):
+// warpgroup 0: warp 0 TMA producer (K, V tiles; Q, dO chunks; the chunk's lse
+// and D rows by bulk copy), warp 1 TMEM owner and MMA issuer; warpgroups 1-2:
+// gradient warps, one warpgroup per half of the chunk's query columns, thread =
+// key row; they also write dK (first) and dV (second) at the end of an item;
+// warpgroup 3: dQ warps, thread = query row, stage dQ_c in shared memory and
 // reduce it into global memory.  All waits are bounded (see sm100.cuh).
 #include <math.h>
 
 #include "nb_internal.h"
+#include "schedule.cuh"
 #include "sm100.cuh"
 #include "warp_mma.cuh"
 
@@ -33,7 +35,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 512;
+
 constexpr int kRows = 128;        // keys per item, queries per chunk
 constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
@@ -66,11 +69,18 @@ struct Cfg {
                        bStg = bDKVFree + 1, bStgFree = bStg + 1, bDone = bStgFree + 1,
                        nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
-  static constexpr int kSmem = oSlot + 16 + 1024;
+  static constexpr int oSched = oSlot + 16;  // work-order prefix table
+  static constexpr int kSmem = oSched + kSchedBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D;
   static constexpr uint32_t tDQ = D == 64 ? 384 : 0;  // for D = 128, dQ reuses the S columns
   static constexpr uint32_t tP = 448;                 // P^T, bf16 pairs (TMEM-P variant)
+  // registers per thread after reallocation: TMA/MMA warpgroup, each gradient
+  // warpgroup, dQ warpgroup (the 16 warps share the 64K-register file)
+  static constexpr int kRegsCtl = D == 64 ? 64 : 40;
+  static constexpr int kRegsGrad = D == 64 ? 176 : 168;
+  static constexpr int kRegsDq = D == 64 ? 96 : 128;
+  static_assert(128 * (kRegsCtl + 2 * kRegsGrad + kRegsDq) <= 65536, "register budget");
 };
 
 struct Params {
@@ -84,13 +94,12 @@ struct Item {
   int b, h, tile, L, I0, nch;
 };
 
-__device__ __forceinline__ Item decode(const Params& p, int it) {
+__device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int tile) {
   const AttnArgs& a = p.a;
   Item x;
-  const int bh = it / p.ntiles;
-  x.tile = it - bh * p.ntiles;
-  x.b = bh / a.heads;
-  x.h = bh - x.b * a.heads;
+  x.b = b;
+  x.h = h;
+  x.tile = tile;
   int L = a.lengths ? a.lengths[x.b] : a.n;
   x.L = min(max(L, 0), a.n);
   const int nb = a.n / kBlock;
@@ -105,19 +114,34 @@ __device__ __forceinline__ Item decode(const Params& p, int it) {
   return x;
 }
 
+// Item `it` of the round-robin order over every tile.
+__device__ __forceinline__ Item decode(const Params& p, int it) {
+  const int bh = it / p.ntiles;
+  const int b = bh / p.a.heads;
+  return decode_bht(p, b, bh - b * p.a.heads, it - bh * p.ntiles);
+}
+
+// Item k of the first pass (non-empty tiles when balanced, else every tile).
+__device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int k) {
+  if (!s.balanced) return decode(p, k);
+  int b, h, tile;
+  sched_nonempty(s, p.a.batch, p.a.heads, k, b, h, tile);
+  return decode_bht(p, b, h, tile);
+}
+
 enum : int { kErrKVFree = 0x31, kErrQDFree, kErrKVFull, kErrQDFull, kErrSDPFree, kErrDQFree,
              kErrPDSFull, kErrDKVFree, kErrGQD, kErrSDPFull, kErrPDSFree, kErrDKVFull,
              kErrDQFull, kErrDone, kErrStg, kErrStgFree };
 
 template <int D>
-__device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tk,
+__device__ int producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tk,
                         const CUtensorMap* tv, const CUtensorMap* tq, const CUtensorMap* tdo) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
   int g = 0, tc = 0;
-  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
-    const Item x = decode(p, it);
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
     if (x.nch == 0) continue;
     const int bh = x.b * a.heads + x.h;
     const int kvb = tc % C::NKV;
@@ -155,7 +179,7 @@ __device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tk,
 }
 
 template <int D>
-__device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
+__device__ int mma_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
   using C = Cfg<D>;
   const uint32_t bar = base + C::oBar;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // K Q^T, V dO^T
@@ -201,8 +225,8 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
     return 0;
   };
   int g = 0, tc = 0, e = 0;
-  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
-    const Item x = decode(p, it);
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
     if (x.nch == 0) continue;
     const int kvb = tc % C::NKV;
     const uint32_t sK = base + C::oK + kvb * 2 * C::kTile, sV = sK + C::kTile;
@@ -240,8 +264,8 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
 
 // Gradient warps: thread = key row r; half hf owns query columns [64 hf, 64 hf + 64).
 template <int D>
-__device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32_t tmem, int wq,
-                          int hf, int lane) {
+__device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
+                          uint32_t tmem, int wq, int hf, int lane) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
@@ -250,17 +274,25 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
   const int nb = a.n / kBlock;
   const float sl2 = a.scale * kLog2e;
   auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
+  // a key tile entirely past its sequence's length: dK = dV = 0 (first group dK, second dV)
+  auto zero_tile = [&](const Item& x) {
+    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
+    const int k = x.tile * kRows + r;
+    if (k < a.n) {
+      uint4* out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(hf == 0 ? a.dk : a.dv) +
+                                            (bh * a.n + k) * D);
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) out[i] = make_uint4(0, 0, 0, 0);
+    }
+  };
   int g = 0, tc = 0;
-  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
-    const Item x = decode(p, it);
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
     const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
     const int k = x.tile * kRows + r;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(hf == 0 ? a.dk : a.dv) + (bh * a.n + k) * D;
     if (x.nch == 0) {  // every key of the tile is padding
-      if (k < a.n) {
-#pragma unroll
-        for (int i = 0; i < D / 8; ++i) reinterpret_cast<uint4*>(out)[i] = make_uint4(0, 0, 0, 0);
-      }
+      zero_tile(x);
       continue;
     }
     const bool row_valid = k < x.L;
@@ -273,19 +305,25 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
       const float* nl = reinterpret_cast<const float*>(gbase + C::oLD + st * 1024);
       const float* Dv = nl + 128;
       uint32_t wp[32], ws[32];  // packed bf16 P^T and dS^T for this thread's 64 queries
+      float sa[2][32], dpa[2][32];
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        tmem_ld32(trow + C::tS + 64 * hf + 32 * jj, sa[jj]);
+        tmem_ld32(trow + C::tDP + 64 * hf + 32 * jj, dpa[jj]);
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        reg_fence(sa[jj]);
+        reg_fence(dpa[jj]);
+      }
+      tc_fence_before();  // S and dP of this chunk are in registers: TMEM may be reused
+      mbar_arrive(bar + 8 * C::bSDPFree);
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
         const int j = 2 * hf + jj;  // 32-query group within the chunk
-        float s[32], dp[32];
-        tmem_ld32(trow + C::tS + 32 * j, s);
-        tmem_ld32(trow + C::tDP + 32 * j, dp);
-        tmem_wait_ld();
-        reg_fence(s);
-        reg_fence(dp);
-        if (jj == 1) {  // S and dP of this chunk are in registers: TMEM may be reused
-          tc_fence_before();
-          mbar_arrive(bar + 8 * C::bSDPFree);
-        }
+        const float(&s)[32] = sa[jj];
+        const float(&dp)[32] = dpa[jj];
         const int qb = x.I0 + 4 * c + j;
         const bool vis = row_valid && qb < nb && abs(qb - kb) <= a.R;
 #pragma unroll
@@ -295,18 +333,20 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
             const float4 n1 = *reinterpret_cast<const float4*>(nl + 32 * j + 8 * cc + 4);
             const float4 d0 = *reinterpret_cast<const float4*>(Dv + 32 * j + 8 * cc);
             const float4 d1 = *reinterpret_cast<const float4*>(Dv + 32 * j + 8 * cc + 4);
-            const float nv[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-            const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-            float pe[8], de[8];
+            const float2 nv[4] = {make_float2(n0.x, n0.y), make_float2(n0.z, n0.w),
+                                  make_float2(n1.x, n1.y), make_float2(n1.z, n1.w)};
+            const float2 nd[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
+                                  make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
+            const float2 sl = make_float2(sl2, sl2);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              pe[e] = ex2_approx(fmaf(s[8 * cc + e], sl2, nv[e]));  // -inf for padding queries -> 0
-              de[e] = pe[e] * (dp[8 * cc + e] - dv[e]);
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              wp[16 * jj + 4 * cc + e] = pack_bf16(pe[2 * e], pe[2 * e + 1]);
-              ws[16 * jj + 4 * cc + e] = pack_bf16(de[2 * e], de[2 * e + 1]);
+            for (int e = 0; e < 4; ++e) {  // pairs of queries, packed fp32x2 arithmetic
+              const float2 x = __ffma2_rn(make_float2(s[8 * cc + 2 * e], s[8 * cc + 2 * e + 1]),
+                                          sl, nv[e]);  // -inf for padding queries -> P = 0
+              const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              const float2 de = __fmul2_rn(
+                  pe, __fadd2_rn(make_float2(dp[8 * cc + 2 * e], dp[8 * cc + 2 * e + 1]), nd[e]));
+              wp[16 * jj + 4 * cc + e] = pack_bf16(pe.x, pe.y);
+              ws[16 * jj + 4 * cc + e] = pack_bf16(de.x, de.y);
             }
           } else {
 #pragma unroll
@@ -365,23 +405,29 @@ __device__ int grad_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32
     g += x.nch;
     ++tc;
   }
+  if (sch.balanced) {  // second pass: the empty key tiles
+    for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+      const Item x = decode(p, it);
+      if (x.nch == 0) zero_tile(x);
+    }
+  }
   return 0;
 }
 
 // dQ warps: thread = query row r of the chunk.
 template <int D>
-__device__ int dq_warps(const Params& p, uint32_t base, uint8_t* gbase, uint32_t tmem, int wq,
-                        int lane, const CUtensorMap* tdq) {
+__device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
+                        uint32_t tmem, int wq, int lane, const CUtensorMap* tdq) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
   const int r = wq * 32 + lane;
   const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-  const bool leader = threadIdx.x == 10 * 32;
+  const bool leader = threadIdx.x == 12 * 32;
   auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
   int g = 0;
-  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
-    const Item x = decode(p, it);
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
     if (x.nch == 0) continue;
     const int bh = x.b * a.heads + x.h;
     for (int c = 0; c < x.nch; ++c) {
@@ -488,12 +534,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDone, 1);
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tk);
-    prefetch_tmap(&tv);
-    prefetch_tmap(&tq);
-    prefetch_tmap(&tdo);
-    prefetch_tmap(&tdq);
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tk);
+      prefetch_tmap(&tv);
+      prefetch_tmap(&tq);
+      prefetch_tmap(&tdo);
+      prefetch_tmap(&tdq);
+    }
+    sched_build(reinterpret_cast<int*>(gbase + C::oSched), p.a, kRows, lane);
   }
   if (warp == 1) {
     tmem_alloc(base + C::oSlot, C::kTmemCols);
@@ -503,28 +552,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + C::oSlot);
+  const Sched sch = sched_view(reinterpret_cast<const int*>(gbase + C::oSched), p.a, p.items);
 
-  int err = 0;
-  if (warp == 0) {
-    if (lane == 0) err = producer<D>(p, base, &tk, &tv, &tq, &tdo);
-  } else if (warp == 1) {
-    if (lane == 0) err = mma_issuer<D>(p, base, tmem);
-  } else if (warp < 10) {
-    err = grad_warps<D>(p, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane);
-  } else {
-    err = dq_warps<D>(p, base, gbase, tmem, warp & 3, lane, &tdq);
-  }
-  if (err) record_error(p.a.err, err);
-
-  __syncthreads();
-  if (warp == 1) {
-    if (lane == 0) {
-      mma_commit(bar + 8 * C::bDone);
-      if (!mbar_wait(bar + 8 * C::bDone, 0)) record_error(p.a.err, kErrDone);
+  // Role branches never join again: each ends with the CTA barrier, after which
+  // warp 1 waits for the tensor cores and frees the TMEM.
+  if (warp < 4) {
+    regs_dec<C::kRegsCtl>();
+    int err = 0;
+    if (warp == 0 && lane == 0) err = producer<D>(p, sch, base, &tk, &tv, &tq, &tdo);
+    if (warp == 1 && lane == 0) err = mma_issuer<D>(p, sch, base, tmem);
+    if (err) record_error(p.a.err, err);
+    __syncthreads();
+    if (warp == 1) {
+      if (lane == 0) {
+        mma_commit(bar + 8 * C::bDone);
+        if (!mbar_wait(bar + 8 * C::bDone, 0)) record_error(p.a.err, kErrDone);
+      }
+      __syncwarp();
+      tc_fence_after();
+      tmem_dealloc(tmem, C::kTmemCols);
     }
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+  } else if (warp < 12) {
+    regs_inc<C::kRegsGrad>();
+    const int err = grad_warps<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
+    if (err) record_error(p.a.err, err);
+    __syncthreads();
+  } else {
+    regs_dec<C::kRegsDq>();
+    const int err = dq_warps<D>(p, sch, base, gbase, tmem, warp & 3, lane, &tdq);
+    if (err) record_error(p.a.err, err);
+    __syncthreads();
   }
 }
 

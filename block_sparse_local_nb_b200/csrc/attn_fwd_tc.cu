@@ -37,6 +37,7 @@
 #include <math.h>
 
 #include "nb_internal.h"
+#include "schedule.cuh"
 #include "sm100.cuh"
 #include "warp_mma.cuh"
 
@@ -76,7 +77,8 @@ struct Cfg {
   // exchange buffers of the two softmax halves: [parity][half][row] fp32
   static constexpr int oXMax = oSlot + 16;
   static constexpr int oXSum = oXMax + 2 * 2 * 128 * 4;
-  static constexpr int kSmem = oXSum + 2 * 2 * 128 * 4 + 1024;  // + slack for 1024-byte alignment
+  static constexpr int oSched = oXSum + 2 * 2 * 128 * 4;  // work-order prefix table
+  static constexpr int kSmem = oSched + kSchedBytes + 1024;  // + slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t tS = 0;    // S buffers: columns [0,128) and [128,256)
   static constexpr uint32_t tO = 256;  // O buffers: [256, 256+D) and [256+D, 256+2D)
@@ -92,13 +94,12 @@ struct Item {
   int b, h, tile, L, J0, nch;
 };
 
-__device__ __forceinline__ Item decode(const Params& p, int it) {
+__device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int tile) {
   const AttnArgs& a = p.a;
   Item x;
-  const int bh = it / p.ntiles;
-  x.tile = it - bh * p.ntiles;
-  x.b = bh / a.heads;
-  x.h = bh - x.b * a.heads;
+  x.b = b;
+  x.h = h;
+  x.tile = tile;
   int L = a.lengths ? a.lengths[x.b] : a.n;
   x.L = min(max(L, 0), a.n);
   const int nb = a.n / kBlock;
@@ -113,18 +114,33 @@ __device__ __forceinline__ Item decode(const Params& p, int it) {
   return x;
 }
 
+// Item `it` of the round-robin order over every tile.
+__device__ __forceinline__ Item decode(const Params& p, int it) {
+  const int bh = it / p.ntiles;
+  const int b = bh / p.a.heads;
+  return decode_bht(p, b, bh - b * p.a.heads, it - bh * p.ntiles);
+}
+
+// Item k of the first pass (non-empty tiles when balanced, else every tile).
+__device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int k) {
+  if (!s.balanced) return decode(p, k);
+  int b, h, tile;
+  sched_nonempty(s, p.a.batch, p.a.heads, k, b, h, tile);
+  return decode_bht(p, b, h, tile);
+}
+
 // error codes: 0x10 + site
 enum : int { kErrQFree = 0x11, kErrKVFree, kErrQFull, kErrKVFull, kErrSFree, kErrOFree, kErrPFull,
              kErrSFull, kErrPFree, kErrPPrev, kErrOFull, kErrDone, kErrXMax, kErrXSum };
 
 template <int D>
-__device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tq,
+__device__ int producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tq,
                         const CUtensorMap* tk, const CUtensorMap* tv) {
   using C = Cfg<D>;
   const uint32_t bar = base + C::oBar;
   int g = 0, tc = 0;
-  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
-    const Item x = decode(p, it);
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
     if (x.nch == 0) continue;
     const int bh = x.b * p.a.heads + x.h;
     const int qs = tc % C::NQ;
@@ -153,7 +169,7 @@ __device__ int producer(const Params& p, uint32_t base, const CUtensorMap* tq,
 }
 
 template <int D>
-__device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
+__device__ int mma_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
   using C = Cfg<D>;
   const uint32_t bar = base + C::oBar;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, kChunk, false, false);  // Q K^T: both K-major
@@ -185,8 +201,8 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
     return 0;
   };
   int g = 0, tc = 0, e = 0;
-  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
-    const Item x = decode(p, it);
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
     if (x.nch == 0) continue;
     const int qs = tc % C::NQ;
     if (!mbar_wait(bar + 8 * (C::bQFull + qs), (tc / C::NQ) & 1)) return kErrQFull;
@@ -216,8 +232,8 @@ __device__ int mma_issuer(const Params& p, uint32_t base, uint32_t tmem) {
 }
 
 template <int D>
-__device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, uint32_t tmem,
-                                int wq, int hf, int lane) {
+__device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
+                                uint32_t tmem, int wq, int hf, int lane) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
@@ -274,19 +290,25 @@ __device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, 
     }
     return 0;
   };
+  // a tile entirely past its sequence's length: O = 0, lse = -inf
+  auto zero_tile = [&](const Item& x) {
+    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
+    const int q = x.tile * kRows + r;
+    if (q < a.n) {
+      uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) +
+                                             (bh * a.n + q) * D + hf * (D / 2));
+#pragma unroll
+      for (int i = 0; i < D / 16; ++i) orow[i] = make_uint4(0, 0, 0, 0);
+      if (a.lse && hf == 0) a.lse[bh * a.n + q] = -INFINITY;
+    }
+  };
   int g = 0, tc = 0, e = 0;
-  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
-    const Item x = decode(p, it);
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
     const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
     const int q = x.tile * kRows + r;
     if (x.nch == 0) {  // the whole tile is padding
-      if (q < a.n) {
-        uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) +
-                                               (bh * a.n + q) * D + hf * (D / 2));
-#pragma unroll
-        for (int i = 0; i < D / 16; ++i) orow[i] = make_uint4(0, 0, 0, 0);
-        if (a.lse && hf == 0) a.lse[bh * a.n + q] = -INFINITY;
-      }
+      zero_tile(x);
       continue;
     }
     const int qb = q / kBlock;
@@ -340,18 +362,19 @@ __device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, 
         m_used = cmax;
       }
       // P = 2^(s scale log2e - m) in bf16 for this half's 64 keys
-      const float nm = -m_used;
+      const float2 nm = make_float2(-m_used, -m_used);
+      const float2 sl = make_float2(sl2, sl2);
       uint32_t w[2][16];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         if (vis[j]) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2_approx(fmaf(s[j][2 * i], sl2, nm));
-            const float p1 = ex2_approx(fmaf(s[j][2 * i + 1], sl2, nm));
-            ls[i & 3] += p0 + p1;
-            w[j][i] = pack_bf16(p0, p1);
+          for (int i = 0; i < 16; ++i) {  // pairs of keys, packed fp32x2 arithmetic
+            const float2 x = __ffma2_rn(make_float2(s[j][2 * i], s[j][2 * i + 1]), sl, nm);
+            const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            ls[i & 1] = __fadd2_rn(ls[i & 1], pv);
+            w[j][i] = pack_bf16(pv.x, pv.y);
           }
         } else {
 #pragma unroll
@@ -379,7 +402,7 @@ __device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, 
         tmem_wait_st();
         l *= alpha;
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
       // this half's 64 keys are exactly slab hf of the 128-byte-swizzled P tile
       uint8_t* prow = gbase + C::oP + pb * C::kPBytes + hf * kSlab + r * 128;
 #pragma unroll
@@ -401,6 +424,12 @@ __device__ int softmax_epilogue(const Params& p, uint32_t base, uint8_t* gbase, 
     ++tc;
   }
   if (pend.valid && (e = epilogue(pend))) return e;
+  if (sch.balanced) {  // second pass: the empty tiles
+    for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+      const Item x = decode(p, it);
+      if (x.nch == 0) zero_tile(x);
+    }
+  }
   return 0;
 }
 
@@ -440,10 +469,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDone, 1);
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tq);
-    prefetch_tmap(&tk);
-    prefetch_tmap(&tv);
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tq);
+      prefetch_tmap(&tk);
+      prefetch_tmap(&tv);
+    }
+    sched_build(reinterpret_cast<int*>(gbase + C::oSched), p.a, kRows, lane);
   }
   if (warp == 1) {
     tmem_alloc(base + C::oSlot, C::kTmemCols);
@@ -453,14 +485,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + C::oSlot);
+  const Sched sch = sched_view(reinterpret_cast<const int*>(gbase + C::oSched), p.a, p.items);
 
   int err = 0;
   if (warp == 0) {
-    if (lane == 0) err = producer<D>(p, base, &tq, &tk, &tv);
+    if (lane == 0) err = producer<D>(p, sch, base, &tq, &tk, &tv);
   } else if (warp == 1) {
-    if (lane == 0) err = mma_issuer<D>(p, base, tmem);
+    if (lane == 0) err = mma_issuer<D>(p, sch, base, tmem);
   } else {
-    err = softmax_epilogue<D>(p, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane);
+    err = softmax_epilogue<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane);
   }
   if (err) record_error(p.a.err, err);
 

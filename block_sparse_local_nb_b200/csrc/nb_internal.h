@@ -40,10 +40,10 @@ bool make_tmap_rows(CUtensorMap* m, const void* base, bool f32, int d, int64_t n
                     int64_t heads_total, int box_cols, int box_rows);
 int num_sms();  // SM count of the current device (cached)
 
-// Backward workspace: [D: rows fp32][-lse*log2(e): rows fp32][dQ accumulator: rows*d fp32],
+// Backward workspace: [-D: rows fp32][-lse*log2(e): rows fp32][dQ accumulator: rows*d fp32],
 // each region 256-byte aligned.
 struct BwdWorkspace {
-  float* D;
+  float* D;      // negated row term -D_i
   float* nlse2;
   float* dqacc;
 };

@@ -59,6 +59,7 @@ struct Cfg {
   static constexpr int NQ = D == 64 ? 2 : 1;   // Q tile buffers
   static constexpr int NKV = D == 64 ? 3 : 2;  // K/V chunk stages
   static constexpr int NP = D == 64 ? 2 : 1;   // P buffers
+  static constexpr int NOB = D == 64 ? 2 : 1;  // O accumulators per half (tiles in flight)
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kKBytes = kChunk * D * 2;
   static constexpr int kPBytes = kRows * kChunk * 2;
@@ -67,21 +68,21 @@ struct Cfg {
   static constexpr int oV = oK + NKV * kKBytes;
   static constexpr int oP = oV + NKV * kKBytes;
   static constexpr int oBar = oP + NP * kPBytes;
-  // barrier indices
+  // barrier indices ([buffer][half] for P, [half][buffer] for O)
   static constexpr int bQFull = 0, bQFree = bQFull + NQ, bKVFull = bQFree + NQ,
                        bKVFree = bKVFull + NKV, bSFull = bKVFree + NKV, bSFree = bSFull + 2,
-                       bPFull = bSFree + 2, bPFree = bPFull + NP, bOFull = bPFree + NP,
-                       bOFree = bOFull + 2, bXMax = bOFree + 2, bXSum = bXMax + 2,
-                       bDone = bXSum + 2, nBar = bDone + 1;
+                       bPFull = bSFree + 2, bPFree = bPFull + 2 * NP, bOFull = bPFree + 2 * NP,
+                       bOFree = bOFull + 2 * NOB, bXSum = bOFree + 2 * NOB, bDone = bXSum + 2,
+                       nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
-  // exchange buffers of the two softmax halves: [parity][half][row] fp32
-  static constexpr int oXMax = oSlot + 16;
-  static constexpr int oXSum = oXMax + 2 * 2 * 128 * 4;
-  static constexpr int oSched = oXSum + 2 * 2 * 128 * 4;  // work-order prefix table
+  // per-tile exchange of the halves' running max and sum: [parity][half][m, l][row] fp32
+  static constexpr int oXSum = oSlot + 16;
+  static constexpr int oSched = oXSum + 2 * 2 * 2 * 128 * 4;  // work-order prefix table
   static constexpr int kSmem = oSched + kSchedBytes + 1024;  // + slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t tS = 0;    // S buffers: columns [0,128) and [128,256)
-  static constexpr uint32_t tO = 256;  // O buffers: [256, 256+D) and [256+D, 256+2D)
+  static constexpr uint32_t tS = 0;  // S buffers: columns [0,128) and [128,256)
+  // O accumulator of half h, buffer ob
+  __device__ static constexpr uint32_t tO(int h, int ob) { return 256 + (h * NOB + ob) * D; }
 };
 
 struct Params {
@@ -173,7 +174,7 @@ __device__ int mma_issuer(const Params& p, const Sched& sch, uint32_t base, uint
   using C = Cfg<D>;
   const uint32_t bar = base + C::oBar;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, kChunk, false, false);  // Q K^T: both K-major
-  constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);       // P V: V is MN-major
+  constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);       // P V: V is MN-major (K = 64 per half)
   // S of chunk G+1 is issued before P V of chunk G, also across items, so the
   // softmax of the next chunk never waits behind a P V product.
   struct Pending {
@@ -182,22 +183,27 @@ __device__ int mma_issuer(const Params& p, const Sched& sch, uint32_t base, uint
     bool last;
   } pend = {false, 0, 0, 0, false};
   auto issue_pv = [&](const Pending& q) -> int {
-    const int st = q.G % C::NKV, pb = q.G % C::NP, ob = q.tc % 2;
-    if (q.c == 0 && !mbar_wait(bar + 8 * (C::bOFree + ob), ((q.tc / 2) & 1) ^ 1)) return kErrOFree;
-    if (!mbar_wait(bar + 8 * (C::bPFull + pb), (q.G / C::NP) & 1)) return kErrPFull;
-    tc_fence_after();
+    const int st = q.G % C::NKV, pb = q.G % C::NP, ob = q.tc % C::NOB;
     const uint32_t sP = base + C::oP + pb * C::kPBytes;
     const uint32_t sV = base + C::oV + st * C::kKBytes;
 #pragma unroll
-    for (int k = 0; k < kChunk / 16; ++k) {
-      const uint64_t ad = smem_desc_sw128(sP + (k >> 2) * kSlab + (k & 3) * 32, 0, 1024);
-      // V is MN-major: 64-column swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
-      mma_bf16_ss(tmem + C::tO + ob * D, ad, smem_desc_sw128(sV + k * 2048, kSlab, 1024), kIdPV,
-                  q.c > 0 || k > 0);
+    for (int h = 0; h < 2; ++h) {  // each half's 64 keys into its own O accumulator
+      if (q.c == 0 &&
+          !mbar_wait(bar + 8 * (C::bOFree + h * C::NOB + ob), ((q.tc / C::NOB) & 1) ^ 1))
+        return kErrOFree;
+      if (!mbar_wait(bar + 8 * (C::bPFull + 2 * pb + h), (q.G / C::NP) & 1)) return kErrPFull;
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        // V is MN-major: 64-column swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
+        mma_bf16_ss(tmem + C::tO(h, ob), smem_desc_sw128(sP + h * kSlab + k * 32, 0, 1024),
+                    smem_desc_sw128(sV + h * 8192 + k * 2048, kSlab, 1024), kIdPV,
+                    q.c > 0 || k > 0);
+      }
+      mma_commit(bar + 8 * (C::bPFree + 2 * pb + h));
+      if (q.last) mma_commit(bar + 8 * (C::bOFull + h * C::NOB + ob));
     }
     mma_commit(bar + 8 * (C::bKVFree + st));
-    mma_commit(bar + 8 * (C::bPFree + pb));
-    if (q.last) mma_commit(bar + 8 * (C::bOFull + ob));
     return 0;
   };
   int g = 0, tc = 0, e = 0;
@@ -241,8 +247,7 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
   const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   const int nb = a.n / kBlock;
   const float sl2 = a.scale * kLog2e;
-  float* xmax = reinterpret_cast<float*>(gbase + C::oXMax);
-  float* xsum = reinterpret_cast<float*>(gbase + C::oXSum);
+  float* xs = reinterpret_cast<float*>(gbase + C::oXSum);
   auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
   // An item's epilogue runs after the next item's first chunk, so the wait for
   // its last P V product overlaps that chunk's softmax.
@@ -250,27 +255,46 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
     bool valid;
     int tc;
     int64_t row;  // global row index of this thread's query (bh * n + q)
-    bool in_range, row_valid;
-    float m, l;   // running max (base 2) and this half's partial sum
-  } pend = {false, 0, 0, false, false, 0.f, 0.f};
+    bool in_range;
+    float m, l;   // this half's running max (base 2) and sum
+  } pend = {false, 0, 0, false, 0.f, 0.f};
+  // Combine the halves: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)).
   auto epilogue = [&](const Epi& x) -> int {
-    const int ob = x.tc % 2, par = x.tc & 1;
-    xsum[(par * 2 + hf) * 128 + r] = x.l;
+    const int ob = x.tc % C::NOB, par = x.tc & 1;
+    xs[((par * 2 + hf) * 2 + 0) * 128 + r] = x.m;
+    xs[((par * 2 + hf) * 2 + 1) * 128 + r] = x.l;
     mbar_arrive(bar + 8 * (C::bXSum + par));
     if (!all_ok(mbar_wait(bar + 8 * (C::bXSum + par), (x.tc >> 1) & 1))) return kErrXSum;
-    const float l = x.l + xsum[(par * 2 + (hf ^ 1)) * 128 + r];
-    if (!all_ok(mbar_wait(bar + 8 * (C::bOFull + ob), (x.tc / 2) & 1))) return kErrOFull;
-    tc_fence_after();
-    float o[D / 64][32];
+    const float mo = xs[((par * 2 + (hf ^ 1)) * 2 + 0) * 128 + r];
+    const float lo = xs[((par * 2 + (hf ^ 1)) * 2 + 1) * 128 + r];
+    const float M = fmaxf(x.m, mo);
+    const float fs = x.m == -INFINITY ? 0.f : ex2_approx(x.m - M);
+    const float fo = mo == -INFINITY ? 0.f : ex2_approx(mo - M);
+    const float L = x.l * fs + lo * fo;
+    const float f0 = hf == 0 ? fs : fo, f1 = hf == 0 ? fo : fs;  // factors of O_0 and O_1
 #pragma unroll
-    for (int j = 0; j < D / 64; ++j) tmem_ld32(trow + C::tO + ob * D + hf * (D / 2) + 32 * j, o[j]);
+    for (int h = 0; h < 2; ++h)
+      if (!all_ok(mbar_wait(bar + 8 * (C::bOFull + h * C::NOB + ob), (x.tc / C::NOB) & 1)))
+        return kErrOFull;
+    tc_fence_after();
+    float o0[D / 64][32], o1[D / 64][32];  // this half's D/2 output columns of O_0 and O_1
+#pragma unroll
+    for (int j = 0; j < D / 64; ++j) {
+      tmem_ld32(trow + C::tO(0, ob) + hf * (D / 2) + 32 * j, o0[j]);
+      tmem_ld32(trow + C::tO(1, ob) + hf * (D / 2) + 32 * j, o1[j]);
+    }
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < D / 64; ++j) reg_fence(o[j]);
+    for (int j = 0; j < D / 64; ++j) {
+      reg_fence(o0[j]);
+      reg_fence(o1[j]);
+    }
     tc_fence_before();
-    mbar_arrive(bar + 8 * (C::bOFree + ob));
-    const bool has = x.row_valid && l > 0.f;
-    const float inv = has ? 1.f / l : 0.f;
+    mbar_arrive(bar + 8 * (C::bOFree + 0 * C::NOB + ob));
+    mbar_arrive(bar + 8 * (C::bOFree + 1 * C::NOB + ob));
+    const bool has = L > 0.f;  // padding rows and rows without a visible key: 0
+    const float inv = has ? 1.f / L : 0.f;
+    const float g0 = f0 * inv, g1 = f1 * inv;
     if (x.in_range) {
       uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) +
                                              x.row * D + hf * (D / 2));
@@ -278,15 +302,14 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
       for (int j = 0; j < D / 64; ++j) {
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          uint4 u;
-          u.x = pack_bf16(o[j][8 * v + 0] * inv, o[j][8 * v + 1] * inv);
-          u.y = pack_bf16(o[j][8 * v + 2] * inv, o[j][8 * v + 3] * inv);
-          u.z = pack_bf16(o[j][8 * v + 4] * inv, o[j][8 * v + 5] * inv);
-          u.w = pack_bf16(o[j][8 * v + 6] * inv, o[j][8 * v + 7] * inv);
-          orow[4 * j + v] = u;
+          float w8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w8[i] = fmaf(o0[j][8 * v + i], g0, o1[j][8 * v + i] * g1);
+          orow[4 * j + v] = make_uint4(pack_bf16(w8[0], w8[1]), pack_bf16(w8[2], w8[3]),
+                                       pack_bf16(w8[4], w8[5]), pack_bf16(w8[6], w8[7]));
         }
       }
-      if (a.lse && hf == 0) a.lse[x.row] = has ? (x.m + log2f(l)) * kLn2 : -INFINITY;
+      if (a.lse && hf == 0) a.lse[x.row] = has ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
     return 0;
   };
@@ -313,9 +336,10 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
     }
     const int qb = q / kBlock;
     const bool row_valid = q < x.L;
+    const int ob = tc % C::NOB;
     float m_used = -INFINITY, l = 0.f;
     for (int c = 0; c < x.nch; ++c) {
-      const int G = g + c, sb = G % 2, pb = G % C::NP, par = G & 1;
+      const int G = g + c, sb = G % 2, pb = G % C::NP;
       if (!all_ok(mbar_wait(bar + 8 * (C::bSFull + sb), (G / 2) & 1))) return kErrSFull;
       tc_fence_after();
       float s[2][32];
@@ -345,13 +369,9 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
           for (int i = 0; i < 32; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[j][i]);
         }
       }
-      float cmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                         fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      // combine with the other half's partial max (raw units; the scale is positive)
-      xmax[(par * 2 + hf) * 128 + r] = cmax;
-      mbar_arrive(bar + 8 * (C::bXMax + par));
-      if (!all_ok(mbar_wait(bar + 8 * (C::bXMax + par), (G >> 1) & 1))) return kErrXMax;
-      cmax = fmaxf(cmax, xmax[(par * 2 + (hf ^ 1)) * 128 + r]) * sl2;
+      // this half's running max (raw scores times the positive scale, base 2)
+      const float cmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * sl2;
       bool need = false;
       float alpha = 1.f;
       if (cmax > m_used + kTau) {
@@ -371,8 +391,8 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
         if (vis[j]) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {  // pairs of keys, packed fp32x2 arithmetic
-            const float2 x = __ffma2_rn(make_float2(s[j][2 * i], s[j][2 * i + 1]), sl, nm);
-            const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            const float2 xv = __ffma2_rn(make_float2(s[j][2 * i], s[j][2 * i + 1]), sl, nm);
+            const float2 pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
             ls[i & 1] = __fadd2_rn(ls[i & 1], pv);
             w[j][i] = pack_bf16(pv.x, pv.y);
           }
@@ -381,16 +401,17 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
           for (int i = 0; i < 16; ++i) w[j][i] = 0u;
         }
       }
-      if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + pb), ((G / C::NP) & 1) ^ 1))) return kErrPFree;
+      if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + 2 * pb + hf), ((G / C::NP) & 1) ^ 1)))
+        return kErrPFree;
       if (__any_sync(0xffffffffu, need)) {
-        // the previous P V product of this tile must have landed before O is rescaled
+        // this half's previous P V product must have landed before its O is rescaled
         const int Gp = G - 1;
-        if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + Gp % C::NP), (Gp / C::NP) & 1)))
+        if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + 2 * (Gp % C::NP) + hf), (Gp / C::NP) & 1)))
           return kErrPPrev;
         tc_fence_after();
-        const uint32_t to = trow + C::tO + (tc % 2) * D + hf * (D / 2);
+        const uint32_t to = trow + C::tO(hf, ob);
 #pragma unroll
-        for (int j = 0; j < D / 64; ++j) {
+        for (int j = 0; j < D / 32; ++j) {
           float ov[32];
           tmem_ld32(to + 32 * j, ov);
           tmem_wait_ld();
@@ -413,13 +434,13 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar + 8 * (C::bPFull + pb));
+      mbar_arrive(bar + 8 * (C::bPFull + 2 * pb + hf));
       if (c == 0 && pend.valid) {  // the previous item's epilogue, deferred past this chunk
         if ((e = epilogue(pend))) return e;
         pend.valid = false;
       }
     }
-    pend = {true, tc, bh * a.n + q, q < a.n, row_valid, m_used, l};
+    pend = {true, tc, bh * a.n + q, q < a.n, m_used, l};
     g += x.nch;
     ++tc;
   }
@@ -457,14 +478,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + 8 * (C::bSFull + i), 1);
       mbar_init(bar + 8 * (C::bSFree + i), 256);
-      mbar_init(bar + 8 * (C::bOFull + i), 1);
-      mbar_init(bar + 8 * (C::bOFree + i), 256);
-      mbar_init(bar + 8 * (C::bXMax + i), 256);
       mbar_init(bar + 8 * (C::bXSum + i), 256);
     }
-    for (int i = 0; i < C::NP; ++i) {
-      mbar_init(bar + 8 * (C::bPFull + i), 256);
+    for (int i = 0; i < 2 * C::NP; ++i) {
+      mbar_init(bar + 8 * (C::bPFull + i), 128);
       mbar_init(bar + 8 * (C::bPFree + i), 1);
+    }
+    for (int i = 0; i < 2 * C::NOB; ++i) {
+      mbar_init(bar + 8 * (C::bOFull + i), 1);
+      mbar_init(bar + 8 * (C::bOFree + i), 256);
     }
     mbar_init(bar + 8 * C::bDone, 1);
     fence_barrier_init();

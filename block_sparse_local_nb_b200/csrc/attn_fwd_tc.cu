@@ -16,21 +16,21 @@
 //              are zero-filled by TMA and masked).
 //   warp 1     TMEM owner and MMA issuer (one thread):
 //                S_c = Q K_c^T   (M 128, N 128, K d)   -> TMEM, two buffers
-//                O  += P_c V_c   (M 128, N d,   K 128) -> TMEM, two buffers
+//                O_h += P_c,h V_c,h  (M 128, N d, K 64; P read from TMEM)
 //              S_{c+1} is issued before P_c V_c so the softmax of the next
 //              chunk overlaps the P V product.
 //   warps 2-9  softmax, two groups of four warps; thread (r, half) owns row r
 //              (TMEM lane r) and 64 of the chunk's 128 key columns.  Per chunk
 //              it reads its 64 scores, masks keys outside its query block's
-//              band or past the length, exchanges the partial row max with the
-//              other half through shared memory, updates the running max and
-//              sum (base 2) and writes P = 2^(s - m) as bf16 into its half of
-//              the shared-memory P tile.  The running output lives in TMEM; it
-//              is rescaled (load, multiply, store; each half its own columns)
-//              only when the row max grows by more than 2^8, otherwise the
-//              stale max is kept (P <= 2^8, exact after the final division).
-//              Epilogue (deferred past the next item's first chunk): the two
-//              partial sums are combined, O / l -> bf16, lse = m + log l.
+//              band or past the length, updates its own running max and sum
+//              (base 2) and writes P = 2^(s - m) as bf16 back into TMEM over
+//              the scores it has read.  Each half keeps its own running output
+//              O_h in TMEM; it is rescaled (load, multiply, store) only when
+//              that half's max grows by more than 2^8, otherwise the stale max
+//              is kept (P <= 2^8, exact after the final division).
+//              Epilogue (deferred past the next item's first chunk): the
+//              halves exchange (m, l) through shared memory and combine
+//              O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / l, lse = M + log l.
 // Every mbarrier wait is bounded; on a timeout the kernel records an error
 // code in the caller-visible error word and tears down (frees TMEM) instead
 // of hanging.
@@ -58,20 +58,17 @@ template <int D>
 struct Cfg {
   static constexpr int NQ = D == 64 ? 2 : 1;   // Q tile buffers
   static constexpr int NKV = D == 64 ? 3 : 2;  // K/V chunk stages
-  static constexpr int NP = D == 64 ? 2 : 1;   // P buffers
   static constexpr int NOB = D == 64 ? 2 : 1;  // O accumulators per half (tiles in flight)
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kKBytes = kChunk * D * 2;
-  static constexpr int kPBytes = kRows * kChunk * 2;
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + NQ * kQBytes;
   static constexpr int oV = oK + NKV * kKBytes;
-  static constexpr int oP = oV + NKV * kKBytes;
-  static constexpr int oBar = oP + NP * kPBytes;
-  // barrier indices ([buffer][half] for P, [half][buffer] for O)
+  static constexpr int oBar = oV + NKV * kKBytes;
+  // barrier indices ([S buffer][half] for P, [half][buffer] for O)
   static constexpr int bQFull = 0, bQFree = bQFull + NQ, bKVFull = bQFree + NQ,
                        bKVFree = bKVFull + NKV, bSFull = bKVFree + NKV, bSFree = bSFull + 2,
-                       bPFull = bSFree + 2, bPFree = bPFull + 2 * NP, bOFull = bPFree + 2 * NP,
+                       bPFull = bSFree + 2, bPVDone = bPFull + 4, bOFull = bPVDone + 4,
                        bOFree = bOFull + 2 * NOB, bXSum = bOFree + 2 * NOB, bDone = bXSum + 2,
                        nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
@@ -80,7 +77,10 @@ struct Cfg {
   static constexpr int oSched = oXSum + 2 * 2 * 2 * 128 * 4;  // work-order prefix table
   static constexpr int kSmem = oSched + kSchedBytes + 1024;  // + slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t tS = 0;  // S buffers: columns [0,128) and [128,256)
+  // S buffers: columns [0,128) and [128,256).  Half h's P (64 keys, two bf16
+  // per column) overwrites the first 32 columns of that half's 64 S columns.
+  static constexpr uint32_t tS = 0;
+  __device__ static constexpr uint32_t tP(int sb, int h) { return tS + sb * kChunk + 64 * h; }
   // O accumulator of half h, buffer ob
   __device__ static constexpr uint32_t tO(int h, int ob) { return 256 + (h * NOB + ob) * D; }
 };
@@ -132,7 +132,7 @@ __device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int 
 
 // error codes: 0x10 + site
 enum : int { kErrQFree = 0x11, kErrKVFree, kErrQFull, kErrKVFull, kErrSFree, kErrOFree, kErrPFull,
-             kErrSFull, kErrPFree, kErrPPrev, kErrOFull, kErrDone, kErrXMax, kErrXSum };
+             kErrSFull, kErrPPrev = 0x1a, kErrOFull, kErrDone, kErrXSum = 0x1e };
 
 template <int D>
 __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tq,
@@ -176,33 +176,35 @@ __device__ int mma_issuer(const Params& p, const Sched& sch, uint32_t base, uint
   constexpr uint32_t kIdS = idesc_bf16_f32(128, kChunk, false, false);  // Q K^T: both K-major
   constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);       // P V: V is MN-major (K = 64 per half)
   // S of chunk G+1 is issued before P V of chunk G, also across items, so the
-  // softmax of the next chunk never waits behind a P V product.
+  // softmax of the next chunk never waits behind a P V product.  P of chunk G
+  // lives in S buffer G % 2, so S of chunk G+2 waits for P V of chunk G.
   struct Pending {
     bool valid;
     int G, c, tc;
     bool last;
   } pend = {false, 0, 0, 0, false};
   auto issue_pv = [&](const Pending& q) -> int {
-    const int st = q.G % C::NKV, pb = q.G % C::NP, ob = q.tc % C::NOB;
-    const uint32_t sP = base + C::oP + pb * C::kPBytes;
+    const int st = q.G % C::NKV, sb = q.G % 2, ob = q.tc % C::NOB;
     const uint32_t sV = base + C::oV + st * C::kKBytes;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {  // each half's 64 keys into its own O accumulator
       if (q.c == 0 &&
           !mbar_wait(bar + 8 * (C::bOFree + h * C::NOB + ob), ((q.tc / C::NOB) & 1) ^ 1))
         return kErrOFree;
-      if (!mbar_wait(bar + 8 * (C::bPFull + 2 * pb + h), (q.G / C::NP) & 1)) return kErrPFull;
+      if (!mbar_wait(bar + 8 * (C::bPFull + 2 * sb + h), (q.G >> 1) & 1)) return kErrPFull;
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        // V is MN-major: 64-column swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
-        mma_bf16_ss(tmem + C::tO(h, ob), smem_desc_sw128(sP + h * kSlab + k * 32, 0, 1024),
+        // P from TMEM (16 keys = 8 columns per step); V is MN-major: 64-column
+        // swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
+        mma_bf16_ts(tmem + C::tO(h, ob), tmem + C::tP(sb, h) + 8 * k,
                     smem_desc_sw128(sV + h * 8192 + k * 2048, kSlab, 1024), kIdPV,
                     q.c > 0 || k > 0);
       }
-      mma_commit(bar + 8 * (C::bPFree + 2 * pb + h));
+      mma_commit(bar + 8 * (C::bPVDone + 2 * sb + h));
       if (q.last) mma_commit(bar + 8 * (C::bOFull + h * C::NOB + ob));
     }
+    mma_commit(bar + 8 * (C::bSFree + sb));
     mma_commit(bar + 8 * (C::bKVFree + st));
     return 0;
   };
@@ -339,7 +341,7 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
     const int ob = tc % C::NOB;
     float m_used = -INFINITY, l = 0.f;
     for (int c = 0; c < x.nch; ++c) {
-      const int G = g + c, sb = G % 2, pb = G % C::NP;
+      const int G = g + c, sb = G % 2;
       if (!all_ok(mbar_wait(bar + 8 * (C::bSFull + sb), (G / 2) & 1))) return kErrSFull;
       tc_fence_after();
       float s[2][32];
@@ -348,8 +350,6 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 2; ++j) reg_fence(s[j]);
-      tc_fence_before();
-      mbar_arrive(bar + 8 * (C::bSFree + sb));
 
       bool vis[2];
       float pm[8];
@@ -384,7 +384,7 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
       // P = 2^(s scale log2e - m) in bf16 for this half's 64 keys
       const float2 nm = make_float2(-m_used, -m_used);
       const float2 sl = make_float2(sl2, sl2);
-      uint32_t w[2][16];
+      uint32_t w[32];  // P of keys 2i, 2i + 1 of this half in w[i]
       float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -394,19 +394,18 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
             const float2 xv = __ffma2_rn(make_float2(s[j][2 * i], s[j][2 * i + 1]), sl, nm);
             const float2 pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
             ls[i & 1] = __fadd2_rn(ls[i & 1], pv);
-            w[j][i] = pack_bf16(pv.x, pv.y);
+            w[16 * j + i] = pack_bf16(pv.x, pv.y);
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[j][i] = 0u;
+          for (int i = 0; i < 16; ++i) w[16 * j + i] = 0u;
         }
       }
-      if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + 2 * pb + hf), ((G / C::NP) & 1) ^ 1)))
-        return kErrPFree;
       if (__any_sync(0xffffffffu, need)) {
         // this half's previous P V product must have landed before its O is rescaled
+        // (need implies c > 0, so chunk G - 1 belongs to this tile)
         const int Gp = G - 1;
-        if (!all_ok(mbar_wait(bar + 8 * (C::bPFree + 2 * (Gp % C::NP) + hf), (Gp / C::NP) & 1)))
+        if (!all_ok(mbar_wait(bar + 8 * (C::bPVDone + 2 * (Gp % 2) + hf), (Gp >> 1) & 1)))
           return kErrPPrev;
         tc_fence_after();
         const uint32_t to = trow + C::tO(hf, ob);
@@ -424,17 +423,11 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
         l *= alpha;
       }
       l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
-      // this half's 64 keys are exactly slab hf of the 128-byte-swizzled P tile
-      uint8_t* prow = gbase + C::oP + pb * C::kPBytes + hf * kSlab + r * 128;
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const int j = c8 >> 2, i0 = (c8 & 3) * 4;
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) =
-            make_uint4(w[j][i0], w[j][i0 + 1], w[j][i0 + 2], w[j][i0 + 3]);
-      }
-      fence_proxy_async_smem();
+      // P over this half's S columns (already read into registers)
+      tmem_st32u(trow + C::tP(sb, hf), w);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar + 8 * (C::bPFull + 2 * pb + hf));
+      mbar_arrive(bar + 8 * (C::bPFull + 2 * sb + hf));
       if (c == 0 && pend.valid) {  // the previous item's epilogue, deferred past this chunk
         if ((e = epilogue(pend))) return e;
         pend.valid = false;
@@ -477,12 +470,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + 8 * (C::bSFull + i), 1);
-      mbar_init(bar + 8 * (C::bSFree + i), 256);
+      mbar_init(bar + 8 * (C::bSFree + i), 1);
       mbar_init(bar + 8 * (C::bXSum + i), 256);
     }
-    for (int i = 0; i < 2 * C::NP; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(bar + 8 * (C::bPFull + i), 128);
-      mbar_init(bar + 8 * (C::bPFree + i), 1);
+      mbar_init(bar + 8 * (C::bPVDone + i), 1);
     }
     for (int i = 0; i < 2 * C::NOB; ++i) {
       mbar_init(bar + 8 * (C::bOFull + i), 1);

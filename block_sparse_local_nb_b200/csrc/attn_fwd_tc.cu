@@ -10,15 +10,17 @@
 // walks the items; consecutive CTAs take neighbouring tiles at the same time,
 // so the key/value blocks their windows share are served from L2.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warp 0     TMA producer: Q tile, then K and V chunks, into 128-byte
 //              swizzled shared memory (3-D tensor maps; rows outside [0, n)
 //              are zero-filled by TMA and masked).
-//   warp 1     TMEM owner and MMA issuer (one thread):
+//   warp 1     TMEM owner and S issuer (one thread):
 //                S_c = Q K_c^T   (M 128, N 128, K d)   -> TMEM, two buffers
+//   warp 10    P V issuer (one thread):
 //                O_h += P_c,h V_c,h  (M 128, N d, K 64; P read from TMEM)
-//              S_{c+1} is issued before P_c V_c so the softmax of the next
-//              chunk overlaps the P V product.
+//              Two issuing threads keep the tensor pipe fed: a lone thread
+//              issuing both streams serialises every wait and commit with
+//              the MMAs.  S_{c+1} is in flight while chunk c's softmax runs.
 //   warps 2-9  softmax, two groups of four warps; thread (r, half) owns row r
 //              (TMEM lane r) and 64 of the chunk's 128 key columns.  Per chunk
 //              it reads its 64 scores, masks keys outside its query block's
@@ -46,7 +48,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kRows = 128;   // query rows per tile
 constexpr int kChunk = 128;  // keys per chunk
 constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 64 bf16
@@ -169,73 +171,79 @@ __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const 
   return 0;
 }
 
+// S = Q K^T for every chunk into S buffer G % 2 (warp 1, one thread).  P of
+// chunk G replaces S in that buffer, so S of chunk G + 2 waits for P V of
+// chunk G, which the other issuer signals on bSFree.
 template <int D>
-__device__ int mma_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
+__device__ int s_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
   using C = Cfg<D>;
   const uint32_t bar = base + C::oBar;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, kChunk, false, false);  // Q K^T: both K-major
-  constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);       // P V: V is MN-major (K = 64 per half)
-  // S of chunk G+1 is issued before P V of chunk G, also across items, so the
-  // softmax of the next chunk never waits behind a P V product.  P of chunk G
-  // lives in S buffer G % 2, so S of chunk G+2 waits for P V of chunk G.
-  struct Pending {
-    bool valid;
-    int G, c, tc;
-    bool last;
-  } pend = {false, 0, 0, 0, false};
-  auto issue_pv = [&](const Pending& q) -> int {
-    const int st = q.G % C::NKV, sb = q.G % 2, ob = q.tc % C::NOB;
-    const uint32_t sV = base + C::oV + st * C::kKBytes;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {  // each half's 64 keys into its own O accumulator
-      if (q.c == 0 &&
-          !mbar_wait(bar + 8 * (C::bOFree + h * C::NOB + ob), ((q.tc / C::NOB) & 1) ^ 1))
-        return kErrOFree;
-      if (!mbar_wait(bar + 8 * (C::bPFull + 2 * sb + h), (q.G >> 1) & 1)) return kErrPFull;
-      tc_fence_after();
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        // P from TMEM (16 keys = 8 columns per step); V is MN-major: 64-column
-        // swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
-        mma_bf16_ts(tmem + C::tO(h, ob), tmem + C::tP(sb, h) + 8 * k,
-                    smem_desc_sw128(sV + h * 8192 + k * 2048, kSlab, 1024), kIdPV,
-                    q.c > 0 || k > 0);
-      }
-      mma_commit(bar + 8 * (C::bPVDone + 2 * sb + h));
-      if (q.last) mma_commit(bar + 8 * (C::bOFull + h * C::NOB + ob));
-    }
-    mma_commit(bar + 8 * (C::bSFree + sb));
-    mma_commit(bar + 8 * (C::bKVFree + st));
-    return 0;
-  };
-  int g = 0, tc = 0, e = 0;
+  int g = 0, tc = 0;
   for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
     const Item x = sched_item(p, sch, it);
     if (x.nch == 0) continue;
     const int qs = tc % C::NQ;
     if (!mbar_wait(bar + 8 * (C::bQFull + qs), (tc / C::NQ) & 1)) return kErrQFull;
-    const uint32_t sQ = base + C::oQ + qs * C::kQBytes;
+    const uint64_t dQ = smem_desc_sw128(base + C::oQ + qs * C::kQBytes, 0, 1024);
     for (int c = 0; c < x.nch; ++c) {
       const int G = g + c, st = G % C::NKV, sb = G % 2;
+      const uint64_t dK = smem_desc_sw128(base + C::oK + st * C::kKBytes, 0, 1024);
+      const uint32_t tD = tmem + C::tS + sb * kChunk;
       if (!mbar_wait(bar + 8 * (C::bKVFull + st), (G / C::NKV) & 1)) return kErrKVFull;
       if (!mbar_wait(bar + 8 * (C::bSFree + sb), ((G / 2) & 1) ^ 1)) return kErrSFree;
       tc_fence_after();
-      const uint32_t sK = base + C::oK + st * C::kKBytes;
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
-        const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
-        mma_bf16_ss(tmem + C::tS + sb * kChunk, smem_desc_sw128(sQ + off, 0, 1024),
-                    smem_desc_sw128(sK + off, 0, 1024), kIdS, k > 0);
+        const uint32_t off = ((k >> 2) * kSlab + (k & 3) * 32) >> 4;  // descriptor address units
+        mma_bf16_ss(tD, dQ + off, dK + off, kIdS, k > 0);
       }
       mma_commit(bar + 8 * (C::bSFull + sb));
       if (c == x.nch - 1) mma_commit(bar + 8 * (C::bQFree + qs));  // the tile's S products issued
-      if (pend.valid && (e = issue_pv(pend))) return e;
-      pend = {true, G, c, tc, c == x.nch - 1};
     }
     g += x.nch;
     ++tc;
   }
-  if (pend.valid && (e = issue_pv(pend))) return e;
+  return 0;
+}
+
+// O_h += P_h V_h for every chunk and half (warp 10, one thread): P from TMEM,
+// V from shared memory.  Completion of chunk G's products frees its S buffer
+// and its K/V stage (S of chunk G completed before its softmax began).
+template <int D>
+__device__ int pv_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
+  using C = Cfg<D>;
+  const uint32_t bar = base + C::oBar;
+  constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);  // V is MN-major (K = 64 per half)
+  int g = 0, tc = 0;
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
+    if (x.nch == 0) continue;
+    const int ob = tc % C::NOB;
+    for (int c = 0; c < x.nch; ++c) {
+      const int G = g + c, st = G % C::NKV, sb = G % 2;
+      // V is MN-major: 64-column swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
+      const uint64_t dV = smem_desc_sw128(base + C::oV + st * C::kKBytes, kSlab, 1024);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // each half's 64 keys into its own O accumulator
+        const uint32_t tO = tmem + C::tO(h, ob), tP = tmem + C::tP(sb, h);
+        if (c == 0 &&
+            !mbar_wait(bar + 8 * (C::bOFree + h * C::NOB + ob), ((tc / C::NOB) & 1) ^ 1))
+          return kErrOFree;
+        if (!mbar_wait(bar + 8 * (C::bPFull + 2 * sb + h), (G >> 1) & 1)) return kErrPFull;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)  // 16 keys = 8 P columns = 2048 bytes of V per step
+          mma_bf16_ts(tO, tP + 8 * k, dV + ((h * 8192 + k * 2048) >> 4), kIdPV, c > 0 || k > 0);
+        mma_commit(bar + 8 * (C::bPVDone + 2 * sb + h));
+        if (c == x.nch - 1) mma_commit(bar + 8 * (C::bOFull + h * C::NOB + ob));
+      }
+      mma_commit(bar + 8 * (C::bSFree + sb));
+      mma_commit(bar + 8 * (C::bKVFree + st));
+    }
+    g += x.nch;
+    ++tc;
+  }
   return 0;
 }
 
@@ -481,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar + 8 * (C::bOFull + i), 1);
       mbar_init(bar + 8 * (C::bOFree + i), 256);
     }
-    mbar_init(bar + 8 * C::bDone, 1);
+    mbar_init(bar + 8 * C::bDone, 2);  // one commit per MMA-issuing thread
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -506,13 +514,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) err = producer<D>(p, sch, base, &tq, &tk, &tv);
   } else if (warp == 1) {
-    if (lane == 0) err = mma_issuer<D>(p, sch, base, tmem);
+    if (lane == 0) err = s_issuer<D>(p, sch, base, tmem);
+  } else if (warp == 10) {
+    if (lane == 0) err = pv_issuer<D>(p, sch, base, tmem);
   } else {
     err = softmax_epilogue<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane);
   }
   if (err) record_error(p.a.err, err);
 
   __syncthreads();
+  if (warp == 10 && lane == 0) mma_commit(bar + 8 * C::bDone);
   if (warp == 1) {
     if (lane == 0) {  // every tensor-core operation of this CTA has completed
       mma_commit(bar + 8 * C::bDone);

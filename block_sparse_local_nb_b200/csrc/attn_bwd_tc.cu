@@ -18,7 +18,9 @@
 //
 // Warp roles (512 threads, four warpgroups with reallocated registers):
 // warpgroup 0: warp 0 TMA producer (K, V tiles; Q, dO chunks; the chunk's lse
-// and D rows by bulk copy), warp 1 TMEM owner and MMA issuer; warpgroups 1-2:
+// and D rows by bulk copy), warp 1 TMEM owner and S/dP issuer, warp 2 issuer of
+// the dV/dK/dQ products (two issuing threads, so neither stream of MMAs waits
+// behind the other's barriers); warpgroups 1-2:
 // gradient warps, one warpgroup per half of the chunk's query columns, thread =
 // key row; they also write dK (first) and dV (second) at the end of an item;
 // warpgroup 3: dQ warps, thread = query row, stage dQ_c in shared memory and
@@ -43,13 +45,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
-  // D = 64: K/V tiles double-buffered; S/dP of chunk G+1 issued before the
-  // dV/dK/dQ products of chunk G (the gradient warps of G+1 then overlap them);
-  // P^T kept in TMEM (64 spare columns) as the A operand of dV, which leaves
-  // room for a dQ staging buffer of its own.
-  // D = 128: TMEM is full (dQ reuses the S columns), so chunks run in order,
-  // P^T goes through shared memory and dQ is staged in the chunk's Q/dO buffer.
-  static constexpr bool kLook = D == 64;
+  // D = 64: K/V tiles double-buffered, three Q/dO stages; P^T kept in TMEM
+  // (64 spare columns) as the A operand of dV, which leaves room for a dQ
+  // staging buffer of its own.
+  // D = 128: TMEM is full (dQ reuses the S columns, so S/dP of chunk G + 1
+  // waits until dQ of chunk G is read out), P^T goes through shared memory
+  // and dQ is staged in the chunk's Q/dO buffer.
   static constexpr bool kPTmem = D == 64;
   static constexpr int NKV = D == 64 ? 2 : 1;  // K/V tile buffers
   static constexpr int NS = D == 64 ? 3 : 1;   // Q/dO chunk stages
@@ -77,7 +78,7 @@ struct Cfg {
   static constexpr uint32_t tP = 448;                 // P^T, bf16 pairs (TMEM-P variant)
   // registers per thread after reallocation: TMA/MMA warpgroup, each gradient
   // warpgroup, dQ warpgroup (the 16 warps share the 64K-register file)
-  static constexpr int kRegsCtl = D == 64 ? 64 : 40;
+  static constexpr int kRegsCtl = D == 64 ? 64 : 48;
   static constexpr int kRegsGrad = D == 64 ? 176 : 168;
   static constexpr int kRegsDq = D == 64 ? 96 : 128;
   static_assert(128 * (kRegsCtl + 2 * kRegsGrad + kRegsDq) <= 65536, "register budget");
@@ -178,87 +179,98 @@ __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const 
   return 0;
 }
 
+// S^T = K Q^T and dP^T = V dO^T for every chunk (warp 1, one thread).  S/dP of
+// chunk G + 1 goes in as soon as the gradient warps hold chunk G's values in
+// registers, so it overlaps their arithmetic and chunk G's gradient products.
 template <int D>
-__device__ int mma_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
+__device__ int sdp_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
   using C = Cfg<D>;
   const uint32_t bar = base + C::oBar;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // K Q^T, V dO^T
-  constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, false, true);    // P^T dO, dS^T Q
-  constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, true, true);      // dS K
-  const uint32_t sP = base + C::oP, sS = base + C::oDS;
-  // The chunk whose dV/dK/dQ products are still to be issued.
-  struct Pending {
-    bool valid;
-    int G, c, st, kvb, tc;
-    bool last;
-  } pend = {false, 0, 0, 0, 0, 0, false};
-  auto issue_grads = [&](const Pending& q) -> int {
-    const uint32_t sQ = base + C::oQ + q.st * 2 * C::kTile, sdO = sQ + C::kTile;
-    const uint32_t sK = base + C::oK + q.kvb * 2 * C::kTile;
-    if (!mbar_wait(bar + 8 * C::bPDSFull, q.G & 1)) return kErrPDSFull;
-    if (q.c == 0 && !mbar_wait(bar + 8 * C::bDKVFree, (q.tc & 1) ^ 1)) return kErrDKVFree;
-    if (D == 64 && !mbar_wait(bar + 8 * C::bDQFree, (q.G & 1) ^ 1)) return kErrDQFree;
-    tc_fence_after();
-#pragma unroll
-    for (int k = 0; k < kRows / 16; ++k) {  // k over the chunk's queries
-      const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
-      if (C::kPTmem)
-        mma_bf16_ts(tmem + C::tDV, tmem + C::tP + 8 * k,
-                    smem_desc_sw128(sdO + k * 2048, kSlab, 1024), kIdKV, q.c > 0 || k > 0);
-      else
-        mma_bf16_ss(tmem + C::tDV, smem_desc_sw128(sP + off, 0, 1024),
-                    smem_desc_sw128(sdO + k * 2048, kSlab, 1024), kIdKV, q.c > 0 || k > 0);
-      mma_bf16_ss(tmem + C::tDK, smem_desc_sw128(sS + off, 0, 1024),
-                  smem_desc_sw128(sQ + k * 2048, kSlab, 1024), kIdKV, q.c > 0 || k > 0);
-    }
-#pragma unroll
-    for (int k = 0; k < kRows / 16; ++k)  // k over the tile's keys
-      mma_bf16_ss(tmem + C::tDQ, smem_desc_sw128(sS + k * 2048, kSlab, 1024),
-                  smem_desc_sw128(sK + k * 2048, kSlab, 1024), kIdQ, k > 0);
-    mma_commit(bar + 8 * C::bPDSFree);
-    mma_commit(bar + 8 * C::bDQFull);
-    if (C::kPTmem) mma_commit(bar + 8 * (C::bQDFree + q.st));  // Q/dO of the chunk consumed
-    if (q.last) {
-      mma_commit(bar + 8 * C::bDKVFull);
-      mma_commit(bar + 8 * (C::bKVFree + q.kvb));
-    }
-    return 0;
-  };
-  int g = 0, tc = 0, e = 0;
+  int g = 0, tc = 0;
   for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
     const Item x = sched_item(p, sch, it);
     if (x.nch == 0) continue;
     const int kvb = tc % C::NKV;
-    const uint32_t sK = base + C::oK + kvb * 2 * C::kTile, sV = sK + C::kTile;
+    const uint32_t sK = base + C::oK + kvb * 2 * C::kTile;
+    const uint64_t dK = smem_desc_sw128(sK, 0, 1024), dV = smem_desc_sw128(sK + C::kTile, 0, 1024);
     if (!mbar_wait(bar + 8 * (C::bKVFull + kvb), (tc / C::NKV) & 1)) return kErrKVFull;
     for (int c = 0; c < x.nch; ++c) {
       const int G = g + c, st = G % C::NS;
-      const uint32_t sQ = base + C::oQ + st * 2 * C::kTile, sdO = sQ + C::kTile;
+      const uint32_t sQ = base + C::oQ + st * 2 * C::kTile;
+      const uint64_t dQ = smem_desc_sw128(sQ, 0, 1024), ddO = smem_desc_sw128(sQ + C::kTile, 0, 1024);
       if (!mbar_wait(bar + 8 * (C::bQDFull + st), (G / C::NS) & 1)) return kErrQDFull;
       if (!mbar_wait(bar + 8 * C::bSDPFree, (G & 1) ^ 1)) return kErrSDPFree;
+      // D = 128: dQ of the previous chunk occupies the S columns until it is read out
       if (D == 128 && !mbar_wait(bar + 8 * C::bDQFree, (G & 1) ^ 1)) return kErrDQFree;
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
-        const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
-        mma_bf16_ss(tmem + C::tS, smem_desc_sw128(sK + off, 0, 1024),
-                    smem_desc_sw128(sQ + off, 0, 1024), kIdS, k > 0);
-        mma_bf16_ss(tmem + C::tDP, smem_desc_sw128(sV + off, 0, 1024),
-                    smem_desc_sw128(sdO + off, 0, 1024), kIdS, k > 0);
+        const uint32_t off = ((k >> 2) * kSlab + (k & 3) * 32) >> 4;  // descriptor address units
+        mma_bf16_ss(tmem + C::tS, desc_add(dK, off), desc_add(dQ, off), kIdS, k > 0);
+        mma_bf16_ss(tmem + C::tDP, desc_add(dV, off), desc_add(ddO, off), kIdS, k > 0);
       }
       mma_commit(bar + 8 * C::bSDPFull);
-      const Pending cur = {true, G, c, st, kvb, tc, c == x.nch - 1};
-      if (C::kLook) {  // lookahead: chunk G-1's products go after S/dP of G
-        if (pend.valid && (e = issue_grads(pend))) return e;
-        pend = cur;
-      } else if ((e = issue_grads(cur))) {  // in order
-        return e;
+    }
+    g += x.nch;
+    ++tc;
+  }
+  return 0;
+}
+
+// dV += P^T dO, dK += dS^T Q and dQ_c = dS K for every chunk (warp 2, one
+// thread).  The S/dP products of a chunk completed before its gradient warps
+// began, so a commit here also covers every read of that chunk's K/V and Q/dO.
+template <int D>
+__device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
+  using C = Cfg<D>;
+  const uint32_t bar = base + C::oBar;
+  constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, false, true);  // P^T dO, dS^T Q
+  constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, true, true);    // dS K
+  const uint64_t dP = smem_desc_sw128(base + C::oP, 0, 1024);
+  const uint64_t dSk = smem_desc_sw128(base + C::oDS, 0, 1024);      // dS^T, K-major A
+  const uint64_t dSm = smem_desc_sw128(base + C::oDS, kSlab, 1024);  // dS, MN-major A
+  int g = 0, tc = 0;
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
+    if (x.nch == 0) continue;
+    const int kvb = tc % C::NKV;
+    const uint64_t dK = smem_desc_sw128(base + C::oK + kvb * 2 * C::kTile, kSlab, 1024);
+    for (int c = 0; c < x.nch; ++c) {
+      const int G = g + c, st = G % C::NS;
+      const uint32_t sQ = base + C::oQ + st * 2 * C::kTile;
+      const uint64_t dQ = smem_desc_sw128(sQ, kSlab, 1024), ddO = smem_desc_sw128(sQ + C::kTile, kSlab, 1024);
+      const bool acc = c > 0;
+      if (!mbar_wait(bar + 8 * C::bPDSFull, G & 1)) return kErrPDSFull;
+      if (c == 0 && !mbar_wait(bar + 8 * C::bDKVFree, (tc & 1) ^ 1)) return kErrDKVFree;
+      if (D == 64 && !mbar_wait(bar + 8 * C::bDQFree, (G & 1) ^ 1)) return kErrDQFree;
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < kRows / 16; ++k) {  // k over the chunk's queries
+        const uint32_t off = ((k >> 2) * kSlab + (k & 3) * 32) >> 4;
+        const uint32_t mn = (k * 2048) >> 4;  // 16 rows of an MN-major operand
+        if (C::kPTmem)
+          mma_bf16_ts(tmem + C::tDV, tmem + C::tP + 8 * k, desc_add(ddO, mn), kIdKV, acc || k > 0);
+        else
+          mma_bf16_ss(tmem + C::tDV, desc_add(dP, off), desc_add(ddO, mn), kIdKV, acc || k > 0);
+        mma_bf16_ss(tmem + C::tDK, desc_add(dSk, off), desc_add(dQ, mn), kIdKV, acc || k > 0);
+      }
+#pragma unroll
+      for (int k = 0; k < kRows / 16; ++k) {  // k over the tile's keys
+        const uint32_t mn = (k * 2048) >> 4;
+        mma_bf16_ss(tmem + C::tDQ, desc_add(dSm, mn), desc_add(dK, mn), kIdQ, k > 0);
+      }
+      mma_commit(bar + 8 * C::bPDSFree);
+      mma_commit(bar + 8 * C::bDQFull);
+      if (C::kPTmem) mma_commit(bar + 8 * (C::bQDFree + st));  // Q/dO of the chunk consumed
+      if (c == x.nch - 1) {
+        mma_commit(bar + 8 * C::bDKVFull);
+        mma_commit(bar + 8 * (C::bKVFree + kvb));
       }
     }
     g += x.nch;
     ++tc;
   }
-  if (pend.valid && (e = issue_grads(pend))) return e;
   return 0;
 }
 
@@ -531,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDKVFree, 256);
     mbar_init(bar + 8 * C::bStg, 128);
     mbar_init(bar + 8 * C::bStgFree, 1);
-    mbar_init(bar + 8 * C::bDone, 1);
+    mbar_init(bar + 8 * C::bDone, 2);  // one commit per MMA-issuing thread
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -560,9 +572,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<C::kRegsCtl>();
     int err = 0;
     if (warp == 0 && lane == 0) err = producer<D>(p, sch, base, &tk, &tv, &tq, &tdo);
-    if (warp == 1 && lane == 0) err = mma_issuer<D>(p, sch, base, tmem);
+    if (warp == 1 && lane == 0) err = sdp_issuer<D>(p, sch, base, tmem);
+    if (warp == 2 && lane == 0) err = grad_issuer<D>(p, sch, base, tmem);
     if (err) record_error(p.a.err, err);
     __syncthreads();
+    if (warp == 2 && lane == 0) mma_commit(bar + 8 * C::bDone);
     if (warp == 1) {
       if (lane == 0) {
         mma_commit(bar + 8 * C::bDone);

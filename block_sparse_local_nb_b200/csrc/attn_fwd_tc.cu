@@ -196,7 +196,7 @@ __device__ int s_issuer(const Params& p, const Sched& sch, uint32_t base, uint32
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = ((k >> 2) * kSlab + (k & 3) * 32) >> 4;  // descriptor address units
-        mma_bf16_ss(tD, dQ + off, dK + off, kIdS, k > 0);
+        mma_bf16_ss(tD, desc_add(dQ, off), desc_add(dK, off), kIdS, k > 0);
       }
       mma_commit(bar + 8 * (C::bSFull + sb));
       if (c == x.nch - 1) mma_commit(bar + 8 * (C::bQFree + qs));  // the tile's S products issued
@@ -234,7 +234,7 @@ __device__ int pv_issuer(const Params& p, const Sched& sch, uint32_t base, uint3
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)  // 16 keys = 8 P columns = 2048 bytes of V per step
-          mma_bf16_ts(tO, tP + 8 * k, dV + ((h * 8192 + k * 2048) >> 4), kIdPV, c > 0 || k > 0);
+          mma_bf16_ts(tO, tP + 8 * k, desc_add(dV, (h * 8192 + k * 2048) >> 4), kIdPV, c > 0 || k > 0);
         mma_commit(bar + 8 * (C::bPVDone + 2 * sb + h));
         if (c == x.nch - 1) mma_commit(bar + 8 * (C::bOFull + h * C::NOB + ob));
       }

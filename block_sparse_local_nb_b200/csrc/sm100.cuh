@@ -242,6 +242,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Descriptor d advanced by `units` 16-byte units (a k-step inside a tile).  The
+// add is a volatile asm so it stays next to the MMA that uses it: otherwise the
+// compiler hoists one 64-bit descriptor per MMA of an unrolled loop out of the
+// chunk loop and the issuing thread runs out of registers.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t units) {
+  uint64_t r;
+  asm volatile("add.s64 %0, %1, %2;" : "=l"(r) : "l"(d), "l"(static_cast<uint64_t>(units)));
+  return r;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B and an fp32 accumulator.
 //   bits 4-5 D format (1 = f32)   bits 7-9 A format (1 = bf16)   bits 10-12 B format
 //   bit 15 A major (0 = K, 1 = MN)   bit 16 B major   bits 17-22 N >> 3   bits 24-28 M >> 4

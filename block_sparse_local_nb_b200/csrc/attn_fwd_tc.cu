@@ -446,10 +446,11 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
     ++tc;
   }
   if (pend.valid && (e = epilogue(pend))) return e;
-  if (sch.balanced) {  // second pass: the empty tiles
-    for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
-      const Item x = decode(p, it);
-      if (x.nch == 0) zero_tile(x);
+  if (sch.balanced) {  // second pass: the empty tiles, listed directly
+    for (int e = blockIdx.x; e < p.items - sch.count; e += gridDim.x) {
+      int b, h, tile;
+      sched_empty(sch, a.batch, a.heads, p.ntiles, e, b, h, tile);
+      zero_tile(decode_bht(p, b, h, tile));
     }
   }
   return 0;

@@ -5,7 +5,8 @@
 // a plain round-robin over all tiles leaves some SMs with many more real tiles
 // than others when lengths vary.  The kernels instead walk the list of
 // non-empty tiles round-robin (every SM gets the same number, +-1), then the
-// list of empty tiles, whose outputs are zero-filled.  The list is implicit: a
+// list of empty tiles, whose outputs are zero-filled (none when every sequence
+// is full length).  The list is implicit: a
 // prefix table over sequences, pre[b] = number of non-empty tiles (all heads)
 // of sequences before b, built once per CTA in shared memory and searched per
 // item.  Batches larger than kMaxSchedBatch fall back to a round-robin over all
@@ -70,6 +71,23 @@ __device__ __forceinline__ void sched_nonempty(const Sched& s, int batch, int he
   const int rem = k - s.pre[b];
   h = rem / T;
   tile = rem - h * T;
+}
+
+// (sequence, head, tile) of item e of the empty list: the tiles of sequence b
+// from ceil(L_b / rows) on, for every head.  Before sequence b there are
+// b * heads * ntiles - pre[b] of them.
+__device__ __forceinline__ void sched_empty(const Sched& s, int batch, int heads, int ntiles, int e,
+                                            int& b, int& h, int& tile) {
+  int lo = 0, hi = batch - 1;  // largest b with epre(b) <= e
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (mid * heads * ntiles - s.pre[mid] <= e) lo = mid; else hi = mid - 1;
+  }
+  b = lo;
+  const int T = (s.pre[b + 1] - s.pre[b]) / heads;  // non-empty tiles per head
+  const int rem = e - (b * heads * ntiles - s.pre[b]);
+  h = rem / (ntiles - T);
+  tile = T + (rem - h * (ntiles - T));
 }
 
 }  // namespace nb

@@ -72,6 +72,7 @@ struct Cfg {
   static constexpr int oSlot = oBar + nBar * 8;
   static constexpr int oSched = oSlot + 16;  // work-order prefix table
   static constexpr int kSmem = oSched + kSchedBytes + 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D;
   static constexpr uint32_t tDQ = D == 64 ? 384 : 0;  // for D = 128, dQ reuses the S columns

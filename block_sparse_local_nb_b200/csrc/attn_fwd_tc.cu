@@ -32,7 +32,9 @@
 //              is kept (P <= 2^8, exact after the final division).
 //              Epilogue (deferred past the next item's first chunk): the
 //              halves exchange (m, l) through shared memory and combine
-//              O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / l, lse = M + log l.
+//              O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / l, lse = M + log l;
+//              the bf16 tile is staged in swizzled shared memory and written
+//              by one TMA tensor store (coalesced, asynchronous).
 // Every mbarrier wait is bounded; on a timeout the kernel records an error
 // code in the caller-visible error word and tears down (frees TMEM) instead
 // of hanging.
@@ -66,7 +68,8 @@ struct Cfg {
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + NQ * kQBytes;
   static constexpr int oV = oK + NKV * kKBytes;
-  static constexpr int oBar = oV + NKV * kKBytes;
+  static constexpr int oStg = oV + NKV * kKBytes;  // output tile staging (D / 64 boxes)
+  static constexpr int oBar = oStg + kRows * D * 2;
   // barrier indices ([S buffer][half] for P, [half][buffer] for O)
   static constexpr int bQFull = 0, bQFree = bQFull + NQ, bKVFull = bQFree + NQ,
                        bKVFree = bKVFull + NKV, bSFull = bKVFree + NKV, bSFree = bSFull + 2,
@@ -78,6 +81,7 @@ struct Cfg {
   static constexpr int oXSum = oSlot + 16;
   static constexpr int oSched = oXSum + 2 * 2 * 2 * 128 * 4;  // work-order prefix table
   static constexpr int kSmem = oSched + kSchedBytes + 1024;  // + slack for 1024-byte alignment
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   static constexpr uint32_t kTmemCols = 512;
   // S buffers: columns [0,128) and [128,256).  Half h's P (64 keys, two bf16
   // per column) overwrites the first 32 columns of that half's 64 S columns.
@@ -249,7 +253,7 @@ __device__ int pv_issuer(const Params& p, const Sched& sch, uint32_t base, uint3
 
 template <int D>
 __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
-                                uint32_t tmem, int wq, int hf, int lane) {
+                                uint32_t tmem, int wq, int hf, int lane, const CUtensorMap* to) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
@@ -263,14 +267,19 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
   // its last P V product overlaps that chunk's softmax.
   struct Epi {
     bool valid;
-    int tc;
+    int tc, bh, tile;
     int64_t row;  // global row index of this thread's query (bh * n + q)
     bool in_range;
     float m, l;   // this half's running max (base 2) and sum
-  } pend = {false, 0, 0, false, 0.f, 0.f};
+  } pend = {false, 0, 0, 0, 0, false, 0.f, 0.f};
+  // One thread stores the staged output tile with TMA; before the staging
+  // buffer is written again it waits until that store has read it.
+  const bool leader = wq == 2 && hf == 0 && lane == 0;
+  uint8_t* stg = gbase + C::oStg;
   // Combine the halves: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)).
   auto epilogue = [&](const Epi& x) -> int {
     const int ob = x.tc % C::NOB, par = x.tc & 1;
+    if (leader) bulk_wait_read0();  // the previous tile's store is done with the staging
     xs[((par * 2 + hf) * 2 + 0) * 128 + r] = x.m;
     xs[((par * 2 + hf) * 2 + 1) * 128 + r] = x.l;
     mbar_arrive(bar + 8 * (C::bXSum + par));
@@ -305,21 +314,27 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
     const bool has = L > 0.f;  // padding rows and rows without a visible key: 0
     const float inv = has ? 1.f / L : 0.f;
     const float g0 = f0 * inv, g1 = f1 * inv;
-    if (x.in_range) {
-      uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) +
-                                             x.row * D + hf * (D / 2));
+    // this half's D / 2 columns = D / 16 chunks of 16 bytes in the swizzled staging
 #pragma unroll
-      for (int j = 0; j < D / 64; ++j) {
+    for (int j = 0; j < D / 64; ++j) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          float w8[8];
+      for (int v = 0; v < 4; ++v) {
+        float w8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w8[i] = fmaf(o0[j][8 * v + i], g0, o1[j][8 * v + i] * g1);
-          orow[4 * j + v] = make_uint4(pack_bf16(w8[0], w8[1]), pack_bf16(w8[2], w8[3]),
-                                       pack_bf16(w8[4], w8[5]), pack_bf16(w8[6], w8[7]));
-        }
+        for (int i = 0; i < 8; ++i) w8[i] = fmaf(o0[j][8 * v + i], g0, o1[j][8 * v + i] * g1);
+        const int gc = hf * (D / 16) + 4 * j + v;  // chunk index within the output row
+        *reinterpret_cast<uint4*>(stg + (gc >> 3) * kSlab + r * 128 + (((gc & 7) ^ (r & 7)) << 4)) =
+            make_uint4(pack_bf16(w8[0], w8[1]), pack_bf16(w8[2], w8[3]), pack_bf16(w8[4], w8[5]),
+                       pack_bf16(w8[6], w8[7]));
       }
-      if (a.lse && hf == 0) a.lse[x.row] = has ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+    if (x.in_range && a.lse && hf == 0) a.lse[x.row] = has ? (M + log2f(L)) * kLn2 : -INFINITY;
+    fence_proxy_async_smem();
+    named_barrier(1, 256);  // the whole tile is staged
+    if (leader) {
+#pragma unroll
+      for (int s = 0; s < D / 64; ++s) tma_store_3d(to, base + C::oStg + s * kSlab, s * 64, x.tile * kRows, x.bh);
+      bulk_commit();
     }
     return 0;
   };
@@ -441,11 +456,12 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
         pend.valid = false;
       }
     }
-    pend = {true, tc, bh * a.n + q, q < a.n, m_used, l};
+    pend = {true, tc, static_cast<int>(bh), x.tile, bh * a.n + q, q < a.n, m_used, l};
     g += x.nch;
     ++tc;
   }
   if (pend.valid && (e = epilogue(pend))) return e;
+  if (leader) bulk_wait_all0();  // the last tile's store has landed before the CTA exits
   if (sch.balanced) {  // second pass: the empty tiles, listed directly
     for (int e = blockIdx.x; e < p.items - sch.count; e += gridDim.x) {
       int b, h, tile;
@@ -459,7 +475,8 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                       const __grid_constant__ CUtensorMap tv, const Params p) {
+                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                       const Params p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -498,6 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tq);
       prefetch_tmap(&tk);
       prefetch_tmap(&tv);
+      prefetch_tmap(&to);
     }
     sched_build(reinterpret_cast<int*>(gbase + C::oSched), p.a, kRows, lane);
   }
@@ -519,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 10) {
     if (lane == 0) err = pv_issuer<D>(p, sch, base, tmem);
   } else {
-    err = softmax_epilogue<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane);
+    err = softmax_epilogue<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane, &to);
   }
   if (err) record_error(p.a.err, err);
 
@@ -540,10 +558,11 @@ template <int D>
 cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg<D>;
   const int64_t heads_total = static_cast<int64_t>(a.batch) * a.heads;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap_bf16_rows(&tq, a.q, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tk, a.k, D, a.n, heads_total, kChunk) ||
-      !make_tmap_bf16_rows(&tv, a.v, D, a.n, heads_total, kChunk))
+      !make_tmap_bf16_rows(&tv, a.v, D, a.n, heads_total, kChunk) ||
+      !make_tmap_bf16_rows(&to, a.o, D, a.n, heads_total, kRows))
     return cudaErrorInvalidValue;
   Params p;
   p.a = a;
@@ -555,7 +574,7 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  attn_fwd_tc_kernel<D><<<grid, kThreads, C::kSmem, stream>>>(tq, tk, tv, p);
+  attn_fwd_tc_kernel<D><<<grid, kThreads, C::kSmem, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 

@@ -61,13 +61,18 @@ struct Cfg {
   static constexpr int oP = oQ + NS * 2 * kTile;  // P^T tile (shared-memory variant only)
   static constexpr int oDS = oP + (kPTmem ? 0 : kPT);
   static constexpr int oStg = oDS + kPT;  // dQ staging box (TMEM-P variant only)
+  // dK and dV tiles are staged for their TMA stores in the P/dS tiles, which
+  // are free once an item's last gradient products have completed
+  static constexpr int oOut = kPTmem ? oDS : oP;
+  static_assert(oDS + kPT - oOut >= 2 * kTile, "dK/dV staging");
   static constexpr int oLD = oStg + (kPTmem ? kSlab : 0);  // stage s: -lse log2e, D
   static constexpr int oBar = oLD + NS * 1024;
   static constexpr int bKVFull = 0, bKVFree = bKVFull + NKV, bQDFull = bKVFree + NKV,
                        bQDFree = bQDFull + NS, bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1,
                        bPDSFull = bSDPFree + 1, bPDSFree = bPDSFull + 1, bDQFull = bPDSFree + 1,
                        bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
-                       bStg = bDKVFree + 1, bStgFree = bStg + 1, bDone = bStgFree + 1,
+                       bStg = bDKVFree + 1, bStgFree = bStg + 1, bOutRead = bStgFree + 1,
+                       bDone = bOutRead + 1,
                        nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
   static constexpr int oSched = oSlot + 16;  // work-order prefix table
@@ -133,7 +138,7 @@ __device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int 
 
 enum : int { kErrKVFree = 0x31, kErrQDFree, kErrKVFull, kErrQDFull, kErrSDPFree, kErrDQFree,
              kErrPDSFull, kErrDKVFree, kErrGQD, kErrSDPFull, kErrPDSFree, kErrDKVFull,
-             kErrDQFull, kErrDone, kErrStg, kErrStgFree };
+             kErrDQFull, kErrDone, kErrStg, kErrStgFree, kErrOutRead };
 
 template <int D>
 __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tk,
@@ -278,7 +283,8 @@ __device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uin
 // Gradient warps: thread = key row r; half hf owns query columns [64 hf, 64 hf + 64).
 template <int D>
 __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
-                          uint32_t tmem, int wq, int hf, int lane) {
+                          uint32_t tmem, int wq, int hf, int lane, const CUtensorMap* tdk,
+                          const CUtensorMap* tdv) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
@@ -287,6 +293,8 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
   const int nb = a.n / kBlock;
   const float sl2 = a.scale * kLog2e;
   auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
+  // one thread issues the dK/dV tile stores and reports when they have read the staging
+  const bool leader = wq == 0 && hf == 0 && lane == 0;
   // a key tile entirely past its sequence's length: dK = dV = 0 (first group dK, second dV)
   auto zero_tile = [&](const Item& x) {
     const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
@@ -303,7 +311,6 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
     const Item x = sched_item(p, sch, it);
     const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
     const int k = x.tile * kRows + r;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(hf == 0 ? a.dk : a.dv) + (bh * a.n + k) * D;
     if (x.nch == 0) {  // every key of the tile is padding
       zero_tile(x);
       continue;
@@ -369,6 +376,13 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
       }
       // the previous chunk's dV/dK/dQ products must be done reading the P/dS tiles
       if (!all_ok(mbar_wait(bar + 8 * C::bPDSFree, (G & 1) ^ 1))) return kErrPDSFree;
+      if (c == 0 && tc > 0) {  // and the previous item's dK/dV stores must have read them
+        if (leader) {
+          bulk_wait_read0();
+          mbar_arrive(bar + 8 * C::bOutRead);
+        }
+        if (!all_ok(mbar_wait(bar + 8 * C::bOutRead, (tc - 1) & 1))) return kErrOutRead;
+      }
       uint8_t* prow = gbase + C::oP + hf * kSlab + r * 128;
       uint8_t* srow = gbase + C::oDS + hf * kSlab + r * 128;
       if (C::kPTmem) {  // this thread's 64 queries = 32 packed columns of P^T in TMEM
@@ -392,32 +406,46 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
       tc_fence_before();
       mbar_arrive(bar + 8 * C::bPDSFull);
     }
-    // epilogue: first group writes dK (times 1/sqrt(d)), second group dV
+    // epilogue: first group stages dK (times 1/sqrt(d)), second group dV, in the
+    // now idle P/dS tiles (128-byte swizzled boxes of 64 columns); one TMA store each
     if (!all_ok(mbar_wait(bar + 8 * C::bDKVFull, tc & 1))) return kErrDKVFull;
     tc_fence_after();
     const float mul = row_valid ? (hf == 0 ? a.scale : 1.f) : 0.f;
     const uint32_t tsrc = trow + (hf == 0 ? C::tDK : C::tDV);
+    uint8_t* stg = gbase + C::oOut + hf * C::kTile + r * 128;
 #pragma unroll
     for (int j = 0; j < D / 32; ++j) {
       float v[32];
       tmem_ld32(tsrc + 32 * j, v);
       tmem_wait_ld();
       reg_fence(v);
-      if (k < a.n) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          reinterpret_cast<uint4*>(out)[4 * j + u] =
-              make_uint4(pack_bf16(v[8 * u] * mul, v[8 * u + 1] * mul),
-                         pack_bf16(v[8 * u + 2] * mul, v[8 * u + 3] * mul),
-                         pack_bf16(v[8 * u + 4] * mul, v[8 * u + 5] * mul),
-                         pack_bf16(v[8 * u + 6] * mul, v[8 * u + 7] * mul));
+      for (int u = 0; u < 4; ++u) {
+        const int gc = 4 * j + u;  // 16-byte chunk of the output row
+        *reinterpret_cast<uint4*>(stg + (gc >> 3) * kSlab + (((gc & 7) ^ (r & 7)) << 4)) =
+            make_uint4(pack_bf16(v[8 * u] * mul, v[8 * u + 1] * mul),
+                       pack_bf16(v[8 * u + 2] * mul, v[8 * u + 3] * mul),
+                       pack_bf16(v[8 * u + 4] * mul, v[8 * u + 5] * mul),
+                       pack_bf16(v[8 * u + 6] * mul, v[8 * u + 7] * mul));
       }
     }
     tc_fence_before();
     mbar_arrive(bar + 8 * C::bDKVFree);
+    fence_proxy_async_smem();
+    named_barrier(1, 256);  // both tiles staged
+    if (leader) {
+#pragma unroll
+      for (int s = 0; s < D / 64; ++s) {
+        tma_store_3d(tdk, base + C::oOut + s * kSlab, s * 64, x.tile * kRows, static_cast<int>(bh));
+        tma_store_3d(tdv, base + C::oOut + C::kTile + s * kSlab, s * 64, x.tile * kRows,
+                     static_cast<int>(bh));
+      }
+      bulk_commit();
+    }
     g += x.nch;
     ++tc;
   }
+  if (leader) bulk_wait_all0();  // the last tiles' stores have landed before the CTA exits
   if (sch.balanced) {  // second pass: the empty tiles, listed directly
     for (int e = blockIdx.x; e < p.items - sch.count; e += gridDim.x) {
       int b, h, tile;
@@ -517,7 +545,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                        const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
-                       const __grid_constant__ CUtensorMap tdq, const Params p) {
+                       const __grid_constant__ CUtensorMap tdq, const __grid_constant__ CUtensorMap tdk,
+                       const __grid_constant__ CUtensorMap tdv, const Params p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -545,6 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDKVFree, 256);
     mbar_init(bar + 8 * C::bStg, 128);
     mbar_init(bar + 8 * C::bStgFree, 1);
+    mbar_init(bar + 8 * C::bOutRead, 1);
     mbar_init(bar + 8 * C::bDone, 2);  // one commit per MMA-issuing thread
     fence_barrier_init();
   }
@@ -555,6 +585,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tq);
       prefetch_tmap(&tdo);
       prefetch_tmap(&tdq);
+      prefetch_tmap(&tdk);
+      prefetch_tmap(&tdv);
     }
     sched_build(reinterpret_cast<int*>(gbase + C::oSched), p.a, kRows, lane);
   }
@@ -590,7 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 12) {
     regs_inc<C::kRegsGrad>();
-    const int err = grad_warps<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
+    const int err =
+        grad_warps<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane, &tdk, &tdv);
     if (err) record_error(p.a.err, err);
     __syncthreads();
   } else {
@@ -608,12 +641,14 @@ cudaError_t launch(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
   Params p;
   p.a = a;
   p.ws = bwd_workspace(a.workspace, rows);
-  CUtensorMap tk, tv, tq, tdo, tdq;
+  CUtensorMap tk, tv, tq, tdo, tdq, tdk, tdv;
   if (!make_tmap_bf16_rows(&tk, a.k, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tv, a.v, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tq, a.q, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tdo, a.dout, D, a.n, heads_total, kRows) ||
-      !make_tmap_rows(&tdq, p.ws.dqacc, true, D, a.n, heads_total, 32, kRows))
+      !make_tmap_rows(&tdq, p.ws.dqacc, true, D, a.n, heads_total, 32, kRows) ||
+      !make_tmap_bf16_rows(&tdk, a.dk, D, a.n, heads_total, kRows) ||
+      !make_tmap_bf16_rows(&tdv, a.dv, D, a.n, heads_total, kRows))
     return cudaErrorInvalidValue;
   p.ntiles = (a.n + kRows - 1) / kRows;
   const int64_t items = heads_total * p.ntiles;
@@ -623,7 +658,7 @@ cudaError_t launch(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  attn_bwd_tc_kernel<D><<<grid, kThreads, C::kSmem, stream>>>(tk, tv, tq, tdo, tdq, p);
+  attn_bwd_tc_kernel<D><<<grid, kThreads, C::kSmem, stream>>>(tk, tv, tq, tdo, tdq, tdk, tdv, p);
   return cudaGetLastError();
 }
 

@@ -20,9 +20,11 @@
 // warpgroup 0: warp 0 TMA producer (K, V tiles; Q, dO chunks; the chunk's lse
 // and D rows by bulk copy), warp 1 TMEM owner and S/dP issuer, warp 2 issuer of
 // the dV/dK/dQ products (two issuing threads, so neither stream of MMAs waits
-// behind the other's barriers); warpgroups 1-2:
+// behind the other's barriers), warp 3 the dK/dV tile stores; warpgroups 1-2:
 // gradient warps, one warpgroup per half of the chunk's query columns, thread =
-// key row; they also write dK (first) and dV (second) at the end of an item;
+// key row; they also stage dK (first) and dV (second) of an item in its K/V
+// buffer, for D = 64 after the next item's first chunk (so the wait for the
+// item's last products overlaps that chunk's arithmetic);
 // warpgroup 3: dQ warps, thread = query row, stage dQ_c in shared memory and
 // reduce it into global memory.  All waits are bounded (see sm100.cuh).
 #include <math.h>
@@ -61,18 +63,17 @@ struct Cfg {
   static constexpr int oP = oQ + NS * 2 * kTile;  // P^T tile (shared-memory variant only)
   static constexpr int oDS = oP + (kPTmem ? 0 : kPT);
   static constexpr int oStg = oDS + kPT;  // dQ staging box (TMEM-P variant only)
-  // dK and dV tiles are staged for their TMA stores in the P/dS tiles, which
-  // are free once an item's last gradient products have completed
-  static constexpr int oOut = kPTmem ? oDS : oP;
-  static_assert(oDS + kPT - oOut >= 2 * kTile, "dK/dV staging");
+  // The dK/dV epilogue of an item is deferred past the next item's first
+  // chunk when the next item's K/V tile has a buffer of its own (D = 64).
+  static constexpr bool kDefer = NKV > 1;
   static constexpr int oLD = oStg + (kPTmem ? kSlab : 0);  // stage s: -lse log2e, D
   static constexpr int oBar = oLD + NS * 1024;
   static constexpr int bKVFull = 0, bKVFree = bKVFull + NKV, bQDFull = bKVFree + NKV,
                        bQDFree = bQDFull + NS, bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1,
                        bPDSFull = bSDPFree + 1, bPDSFree = bPDSFull + 1, bDQFull = bPDSFree + 1,
                        bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
-                       bStg = bDKVFree + 1, bStgFree = bStg + 1, bOutRead = bStgFree + 1,
-                       bDone = bOutRead + 1,
+                       bStg = bDKVFree + 1, bStgFree = bStg + 1, bOutFull = bStgFree + 1,
+                       bDone = bOutFull + NKV,
                        nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
   static constexpr int oSched = oSlot + 16;  // work-order prefix table
@@ -138,7 +139,7 @@ __device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int 
 
 enum : int { kErrKVFree = 0x31, kErrQDFree, kErrKVFull, kErrQDFull, kErrSDPFree, kErrDQFree,
              kErrPDSFull, kErrDKVFree, kErrGQD, kErrSDPFull, kErrPDSFree, kErrDKVFull,
-             kErrDQFull, kErrDone, kErrStg, kErrStgFree, kErrOutRead };
+             kErrDQFull, kErrDone, kErrStg, kErrStgFree, kErrOutFull };
 
 template <int D>
 __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tk,
@@ -226,7 +227,7 @@ __device__ int sdp_issuer(const Params& p, const Sched& sch, uint32_t base, uint
 
 // dV += P^T dO, dK += dS^T Q and dQ_c = dS K for every chunk (warp 2, one
 // thread).  The S/dP products of a chunk completed before its gradient warps
-// began, so a commit here also covers every read of that chunk's K/V and Q/dO.
+// began, so a commit here also covers every read of that chunk's Q/dO.
 template <int D>
 __device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
   using C = Cfg<D>;
@@ -269,10 +270,7 @@ __device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uin
       mma_commit(bar + 8 * C::bPDSFree);
       mma_commit(bar + 8 * C::bDQFull);
       if (C::kPTmem) mma_commit(bar + 8 * (C::bQDFree + st));  // Q/dO of the chunk consumed
-      if (c == x.nch - 1) {
-        mma_commit(bar + 8 * C::bDKVFull);
-        mma_commit(bar + 8 * (C::bKVFree + kvb));
-      }
+      if (c == x.nch - 1) mma_commit(bar + 8 * C::bDKVFull);
     }
     g += x.nch;
     ++tc;
@@ -280,11 +278,40 @@ __device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uin
   return 0;
 }
 
+// dK/dV tile stores (warp 3, one thread).  The gradient warps stage an item's
+// dK and dV in the item's own K and V buffers (free once its last products
+// have completed); the buffer is handed back to the producer once the stores
+// have read it.
+template <int D>
+__device__ int out_storer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tdk,
+                          const CUtensorMap* tdv) {
+  using C = Cfg<D>;
+  const uint32_t bar = base + C::oBar;
+  int tc = 0;
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
+    if (x.nch == 0) continue;
+    const int kvb = tc % C::NKV, bh = x.b * p.a.heads + x.h;
+    const uint32_t sk = base + C::oK + kvb * 2 * C::kTile;
+    if (!mbar_wait(bar + 8 * (C::bOutFull + kvb), (tc / C::NKV) & 1)) return kErrOutFull;
+#pragma unroll
+    for (int s = 0; s < D / 64; ++s) {
+      tma_store_3d(tdk, sk + s * kSlab, s * 64, x.tile * kRows, bh);
+      tma_store_3d(tdv, sk + C::kTile + s * kSlab, s * 64, x.tile * kRows, bh);
+    }
+    bulk_commit();
+    bulk_wait_read0();
+    mbar_arrive(bar + 8 * (C::bKVFree + kvb));
+    ++tc;
+  }
+  bulk_wait_all0();  // the stores have landed before the CTA exits
+  return 0;
+}
+
 // Gradient warps: thread = key row r; half hf owns query columns [64 hf, 64 hf + 64).
 template <int D>
 __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
-                          uint32_t tmem, int wq, int hf, int lane, const CUtensorMap* tdk,
-                          const CUtensorMap* tdv) {
+                          uint32_t tmem, int wq, int hf, int lane) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
@@ -293,8 +320,43 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
   const int nb = a.n / kBlock;
   const float sl2 = a.scale * kLog2e;
   auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
-  // one thread issues the dK/dV tile stores and reports when they have read the staging
-  const bool leader = wq == 0 && hf == 0 && lane == 0;
+  // Epilogue: this thread's row of dK (first group, times 1/sqrt(d)) or dV
+  // (second group) as packed bf16, then into the item's K (dK) or V (dV)
+  // buffer as 128-byte swizzled boxes for the tile stores.
+  uint32_t outp[D / 2];
+  auto epi_load = [&](int etc, bool erow_valid) -> int {
+    if (!all_ok(mbar_wait(bar + 8 * C::bDKVFull, etc & 1))) return kErrDKVFull;
+    tc_fence_after();
+    const float mul = erow_valid ? (hf == 0 ? a.scale : 1.f) : 0.f;
+    const uint32_t tsrc = trow + (hf == 0 ? C::tDK : C::tDV);
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) {
+      float v[32];
+      tmem_ld32(tsrc + 32 * j, v);
+      tmem_wait_ld();
+      reg_fence(v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) outp[16 * j + i] = pack_bf16(v[2 * i] * mul, v[2 * i + 1] * mul);
+    }
+    tc_fence_before();
+    mbar_arrive(bar + 8 * C::bDKVFree);
+    return 0;
+  };
+  auto epi_stage = [&](int ekvb) {
+    uint8_t* stg = gbase + C::oK + ekvb * 2 * C::kTile + hf * C::kTile + r * 128;
+#pragma unroll
+    for (int gc = 0; gc < D / 8; ++gc)  // 16-byte chunk of the output row
+      *reinterpret_cast<uint4*>(stg + (gc >> 3) * kSlab + (((gc & 7) ^ (r & 7)) << 4)) =
+          make_uint4(outp[4 * gc], outp[4 * gc + 1], outp[4 * gc + 2], outp[4 * gc + 3]);
+    fence_proxy_async_smem();
+    mbar_arrive(bar + 8 * (C::bOutFull + ekvb));
+  };
+  struct Pend {
+    bool valid;
+    int tc;
+    bool row_valid;
+  } pend = {false, 0, false};
+  int e = 0;
   // a key tile entirely past its sequence's length: dK = dV = 0 (first group dK, second dV)
   auto zero_tile = [&](const Item& x) {
     const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
@@ -309,7 +371,6 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
   int g = 0, tc = 0;
   for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
     const Item x = sched_item(p, sch, it);
-    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
     const int k = x.tile * kRows + r;
     if (x.nch == 0) {  // every key of the tile is padding
       zero_tile(x);
@@ -376,13 +437,7 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
       }
       // the previous chunk's dV/dK/dQ products must be done reading the P/dS tiles
       if (!all_ok(mbar_wait(bar + 8 * C::bPDSFree, (G & 1) ^ 1))) return kErrPDSFree;
-      if (c == 0 && tc > 0) {  // and the previous item's dK/dV stores must have read them
-        if (leader) {
-          bulk_wait_read0();
-          mbar_arrive(bar + 8 * C::bOutRead);
-        }
-        if (!all_ok(mbar_wait(bar + 8 * C::bOutRead, (tc - 1) & 1))) return kErrOutRead;
-      }
+
       uint8_t* prow = gbase + C::oP + hf * kSlab + r * 128;
       uint8_t* srow = gbase + C::oDS + hf * kSlab + r * 128;
       if (C::kPTmem) {  // this thread's 64 queries = 32 packed columns of P^T in TMEM
@@ -405,47 +460,27 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar + 8 * C::bPDSFull);
-    }
-    // epilogue: first group stages dK (times 1/sqrt(d)), second group dV, in the
-    // now idle P/dS tiles (128-byte swizzled boxes of 64 columns); one TMA store each
-    if (!all_ok(mbar_wait(bar + 8 * C::bDKVFull, tc & 1))) return kErrDKVFull;
-    tc_fence_after();
-    const float mul = row_valid ? (hf == 0 ? a.scale : 1.f) : 0.f;
-    const uint32_t tsrc = trow + (hf == 0 ? C::tDK : C::tDV);
-    uint8_t* stg = gbase + C::oOut + hf * C::kTile + r * 128;
-#pragma unroll
-    for (int j = 0; j < D / 32; ++j) {
-      float v[32];
-      tmem_ld32(tsrc + 32 * j, v);
-      tmem_wait_ld();
-      reg_fence(v);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int gc = 4 * j + u;  // 16-byte chunk of the output row
-        *reinterpret_cast<uint4*>(stg + (gc >> 3) * kSlab + (((gc & 7) ^ (r & 7)) << 4)) =
-            make_uint4(pack_bf16(v[8 * u] * mul, v[8 * u + 1] * mul),
-                       pack_bf16(v[8 * u + 2] * mul, v[8 * u + 3] * mul),
-                       pack_bf16(v[8 * u + 4] * mul, v[8 * u + 5] * mul),
-                       pack_bf16(v[8 * u + 6] * mul, v[8 * u + 7] * mul));
+      if (C::kDefer && c == 0 && pend.valid) {
+        // the previous item's epilogue: its last products completed before the
+        // P/dS tiles were free, so only the TMEM read delays this chunk's products
+        if ((e = epi_load(pend.tc, pend.row_valid))) return e;
+        epi_stage(pend.tc % C::NKV);
+        pend.valid = false;
       }
     }
-    tc_fence_before();
-    mbar_arrive(bar + 8 * C::bDKVFree);
-    fence_proxy_async_smem();
-    named_barrier(1, 256);  // both tiles staged
-    if (leader) {
-#pragma unroll
-      for (int s = 0; s < D / 64; ++s) {
-        tma_store_3d(tdk, base + C::oOut + s * kSlab, s * 64, x.tile * kRows, static_cast<int>(bh));
-        tma_store_3d(tdv, base + C::oOut + C::kTile + s * kSlab, s * 64, x.tile * kRows,
-                     static_cast<int>(bh));
-      }
-      bulk_commit();
+    if (C::kDefer) {
+      pend = {true, tc, row_valid};
+    } else {
+      if ((e = epi_load(tc, row_valid))) return e;
+      epi_stage(tc % C::NKV);
     }
     g += x.nch;
     ++tc;
   }
-  if (leader) bulk_wait_all0();  // the last tiles' stores have landed before the CTA exits
+  if (C::kDefer && pend.valid) {
+    if ((e = epi_load(pend.tc, pend.row_valid))) return e;
+    epi_stage(pend.tc % C::NKV);
+  }
   if (sch.balanced) {  // second pass: the empty tiles, listed directly
     for (int e = blockIdx.x; e < p.items - sch.count; e += gridDim.x) {
       int b, h, tile;
@@ -574,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDKVFree, 256);
     mbar_init(bar + 8 * C::bStg, 128);
     mbar_init(bar + 8 * C::bStgFree, 1);
-    mbar_init(bar + 8 * C::bOutRead, 1);
+    for (int i = 0; i < C::NKV; ++i) mbar_init(bar + 8 * (C::bOutFull + i), 256);
     mbar_init(bar + 8 * C::bDone, 2);  // one commit per MMA-issuing thread
     fence_barrier_init();
   }
@@ -608,6 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) err = producer<D>(p, sch, base, &tk, &tv, &tq, &tdo);
     if (warp == 1 && lane == 0) err = sdp_issuer<D>(p, sch, base, tmem);
     if (warp == 2 && lane == 0) err = grad_issuer<D>(p, sch, base, tmem);
+    if (warp == 3 && lane == 0) err = out_storer<D>(p, sch, base, &tdk, &tdv);
     if (err) record_error(p.a.err, err);
     __syncthreads();
     if (warp == 2 && lane == 0) mma_commit(bar + 8 * C::bDone);
@@ -622,8 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 12) {
     regs_inc<C::kRegsGrad>();
-    const int err =
-        grad_warps<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane, &tdk, &tdv);
+    const int err = grad_warps<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
     if (err) record_error(p.a.err, err);
     __syncthreads();
   } else {

@@ -21,6 +21,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int D>
 __global__ void __launch_bounds__(256) bwd_rowterm_kernel(AttnArgs a, int64_t rows) {
   constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
+  pdl_trigger();
+  pdl_wait();
   const BwdWorkspace w = bwd_workspace(a.workspace, rows);
   const int64_t gt = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t row = gt / TPR;
@@ -65,6 +67,8 @@ __global__ void __launch_bounds__(256) bwd_rowterm_kernel(AttnArgs a, int64_t ro
 
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dq_out_kernel(AttnArgs a, int64_t rows) {
+  pdl_trigger();
+  pdl_wait();
   const float* dqacc = bwd_workspace(a.workspace, rows).dqacc;
   const int64_t nvec = rows * D / 8;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nvec;
@@ -94,7 +98,8 @@ cudaError_t run(const AttnArgs& a, cudaStream_t stream) {
   {
     const int64_t threads = rows * (D / 8);
     const int64_t blocks = (threads + 255) / 256;
-    bwd_rowterm_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(a, rows);
+    cudaError_t e = launch_pdl(bwd_rowterm_kernel<D>, dim3((unsigned)blocks), dim3(256), 0, stream, a, rows);
+    if (e != cudaSuccess) return e;
   }
   cudaError_t e = launch_bwd_main_tc(a, rows, stream);
   if (e != cudaSuccess) return e;
@@ -102,9 +107,9 @@ cudaError_t run(const AttnArgs& a, cudaStream_t stream) {
     const int64_t nvec = rows * D / 8;
     int64_t blocks = (nvec + 255) / 256;
     if (blocks > 148 * 64) blocks = 148 * 64;
-    bwd_dq_out_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(a, rows);
+    e = launch_pdl(bwd_dq_out_kernel<D>, dim3((unsigned)blocks), dim3(256), 0, stream, a, rows);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace

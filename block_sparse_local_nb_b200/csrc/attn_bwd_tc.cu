@@ -623,12 +623,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tdk);
       prefetch_tmap(&tdv);
     }
-    sched_build(reinterpret_cast<int*>(gbase + C::oSched), p.a, kRows, lane);
   }
   if (warp == 1) {
     tmem_alloc(base + C::oSlot, C::kTmemCols);
     tmem_relinquish();
   }
+  pdl_wait();  // everything above overlaps the previous kernel's tail
+  if (warp == 0) sched_build(reinterpret_cast<int*>(gbase + C::oSched), p.a, kRows, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -645,6 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 2 && lane == 0) err = grad_issuer<D>(p, sch, base, tmem);
     if (warp == 3 && lane == 0) err = out_storer<D>(p, sch, base, &tdk, &tdv);
     if (err) record_error(p.a.err, err);
+    pdl_trigger();  // this CTA's work is issued: the next kernel may start launching
     __syncthreads();
     if (warp == 2 && lane == 0) mma_commit(bar + 8 * C::bDone);
     if (warp == 1) {
@@ -660,11 +662,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_inc<C::kRegsGrad>();
     const int err = grad_warps<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
     if (err) record_error(p.a.err, err);
+    pdl_trigger();  // this CTA's work is issued: the next kernel may start launching
     __syncthreads();
   } else {
     regs_dec<C::kRegsDq>();
     const int err = dq_warps<D>(p, sch, base, gbase, tmem, warp & 3, lane, &tdq);
     if (err) record_error(p.a.err, err);
+    pdl_trigger();  // this CTA's work is issued: the next kernel may start launching
     __syncthreads();
   }
 }
@@ -693,8 +697,8 @@ cudaError_t launch(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  attn_bwd_tc_kernel<D><<<grid, kThreads, C::kSmem, stream>>>(tk, tv, tq, tdo, tdq, tdk, tdv, p);
-  return cudaGetLastError();
+  return launch_pdl(attn_bwd_tc_kernel<D>, dim3(grid), dim3(kThreads), C::kSmem, stream, tk, tv, tq,
+                    tdo, tdq, tdk, tdv, p);
 }
 
 }  // namespace

@@ -517,12 +517,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tv);
       prefetch_tmap(&to);
     }
-    sched_build(reinterpret_cast<int*>(gbase + C::oSched), p.a, kRows, lane);
   }
   if (warp == 1) {
     tmem_alloc(base + C::oSlot, C::kTmemCols);
     tmem_relinquish();
   }
+  pdl_wait();  // everything above overlaps the previous kernel's tail
+  if (warp == 0) sched_build(reinterpret_cast<int*>(gbase + C::oSched), p.a, kRows, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -541,6 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (err) record_error(p.a.err, err);
 
+  pdl_trigger();  // this CTA's work is issued: the next kernel may start launching
   __syncthreads();
   if (warp == 10 && lane == 0) mma_commit(bar + 8 * C::bDone);
   if (warp == 1) {
@@ -574,8 +576,8 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  attn_fwd_tc_kernel<D><<<grid, kThreads, C::kSmem, stream>>>(tq, tk, tv, to, p);
-  return cudaGetLastError();
+  return launch_pdl(attn_fwd_tc_kernel<D>, dim3(grid), dim3(kThreads), C::kSmem, stream, tq, tk, tv,
+                    to, p);
 }
 
 }  // namespace

@@ -57,6 +57,33 @@ __host__ __device__ inline BwdWorkspace bwd_workspace(void* ws, int64_t rows) {
 }
 cudaError_t launch_bwd_main_tc(const AttnArgs& a, int64_t rows, cudaStream_t stream);
 
+// Programmatic dependent launch.  Every kernel of this library is launched
+// with it: a kernel may begin (set up barriers, tensor memory, descriptor
+// prefetches) while the previous kernel on the stream is finishing, and
+// executes pdl_wait() in every thread before its first access to global memory
+// that earlier work on the stream may write or read.  pdl_trigger() lets the
+// next kernel launch early; it never orders memory.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 cudaError_t launch_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
                                  int k, cudaStream_t stream);
 cudaError_t launch_attn_fwd_f32(const AttnArgs& a, cudaStream_t stream);

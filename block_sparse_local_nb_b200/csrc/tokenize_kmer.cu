@@ -72,6 +72,8 @@ __global__ void __launch_bounds__(256) tokenize_kmer_kernel(const uint8_t* __res
                                                             uint8_t* __restrict__ packed,
                                                             int64_t nchunks, bool ids_vec,
                                                             bool packed_vec) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t nwin = len - K + 1;  // number of windows (may be <= 0)
   const int64_t npacked = (len + 3) >> 2;
   for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < nchunks;
@@ -137,14 +139,14 @@ __global__ void __launch_bounds__(256) tokenize_kmer_kernel(const uint8_t* __res
 }
 
 template <int K>
-void launch_k(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed, int64_t nchunks,
-              unsigned blocks, bool aligned, bool ids_vec, bool packed_vec, cudaStream_t stream) {
+cudaError_t launch_k(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
+                     int64_t nchunks, unsigned blocks, bool aligned, bool ids_vec, bool packed_vec,
+                     cudaStream_t stream) {
   if (aligned)
-    tokenize_kmer_kernel<K, true>
-        <<<blocks, 256, 0, stream>>>(seq, len, ids, packed, nchunks, ids_vec, packed_vec);
-  else
-    tokenize_kmer_kernel<K, false>
-        <<<blocks, 256, 0, stream>>>(seq, len, ids, packed, nchunks, ids_vec, packed_vec);
+    return launch_pdl(tokenize_kmer_kernel<K, true>, dim3(blocks), dim3(256), 0, stream, seq, len,
+                      ids, packed, nchunks, ids_vec, packed_vec);
+  return launch_pdl(tokenize_kmer_kernel<K, false>, dim3(blocks), dim3(256), 0, stream, seq, len,
+                    ids, packed, nchunks, ids_vec, packed_vec);
 }
 
 }  // namespace
@@ -161,15 +163,14 @@ cudaError_t launch_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids,
   const bool packed_vec = (reinterpret_cast<uintptr_t>(packed) & 7u) == 0;
   const unsigned b = static_cast<unsigned>(blocks);
   switch (k) {
-    case 1: launch_k<1>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream); break;
-    case 2: launch_k<2>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream); break;
-    case 3: launch_k<3>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream); break;
-    case 4: launch_k<4>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream); break;
-    case 5: launch_k<5>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream); break;
-    case 6: launch_k<6>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream); break;
-    default: launch_k<7>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream); break;
+    case 1: return launch_k<1>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream);
+    case 2: return launch_k<2>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream);
+    case 3: return launch_k<3>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream);
+    case 4: return launch_k<4>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream);
+    case 5: return launch_k<5>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream);
+    case 6: return launch_k<6>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream);
+    default: return launch_k<7>(seq, len, ids, packed, nchunks, b, aligned, ids_vec, packed_vec, stream);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace nb

@@ -106,6 +106,30 @@ def test_bf16_dk_dv_deterministic():
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
 
 
+def test_bf16_chained_calls_without_sync_match_synchronized():
+    """Kernels start early (programmatic dependent launch) but wait for the
+    previous kernel before touching memory: a chain in which each call
+    consumes the previous call's outputs gives the same bits with or without
+    a device synchronisation between the calls."""
+    q, k, v, do = _cuda(*random_attn_inputs(2, 4, 1024, 64, "bf16", seed=21))
+    L = _lengths([1024, 613])
+
+    def chain(sync):
+        o, lse = run_fwd(q, k, v, L, 2)
+        sync()
+        _, dk, dv = run_bwd(q, k, v, o, do, lse, L, 2)
+        sync()
+        o2, lse2 = run_fwd(dk, dv, k, L, 2)  # reads what the last kernel just wrote
+        sync()
+        return o, lse, dk, dv, o2, lse2
+
+    a = chain(lambda: None)
+    b = chain(torch.cuda.synchronize)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
 def test_bf16_padding_contents_are_ignored():
     """Garbage (1e4) in Q, K, V and dO past each length changes nothing."""
     n, R, d = 640, 2, 64

@@ -358,15 +358,13 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
   } pend = {false, 0, false};
   int e = 0;
   // a key tile entirely past its sequence's length: dK = dV = 0 (first group dK, second dV)
+  // (the tile's rows are contiguous: each group stores it as one coalesced run)
   auto zero_tile = [&](const Item& x) {
-    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
-    const int k = x.tile * kRows + r;
-    if (k < a.n) {
-      uint4* out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(hf == 0 ? a.dk : a.dv) +
-                                            (bh * a.n + k) * D);
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i) out[i] = make_uint4(0, 0, 0, 0);
-    }
+    const int64_t row0 = (static_cast<int64_t>(x.b) * a.heads + x.h) * a.n + x.tile * kRows;
+    const int rows = min(kRows, a.n - x.tile * kRows);
+    uint4* out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(hf == 0 ? a.dk : a.dv) +
+                                          row0 * D);
+    for (int i = r; i < rows * (D / 8); i += 128) out[i] = make_uint4(0, 0, 0, 0);
   };
   int g = 0, tc = 0;
   for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {

@@ -339,16 +339,14 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
     return 0;
   };
   // a tile entirely past its sequence's length: O = 0, lse = -inf
+  // (the tile's rows are contiguous: the 256 threads store it as one coalesced run)
   auto zero_tile = [&](const Item& x) {
-    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
-    const int q = x.tile * kRows + r;
-    if (q < a.n) {
-      uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) +
-                                             (bh * a.n + q) * D + hf * (D / 2));
-#pragma unroll
-      for (int i = 0; i < D / 16; ++i) orow[i] = make_uint4(0, 0, 0, 0);
-      if (a.lse && hf == 0) a.lse[bh * a.n + q] = -INFINITY;
-    }
+    const int64_t row0 = (static_cast<int64_t>(x.b) * a.heads + x.h) * a.n + x.tile * kRows;
+    const int rows = min(kRows, a.n - x.tile * kRows);
+    uint4* out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(const_cast<void*>(a.o)) +
+                                          row0 * D);
+    for (int i = hf * 128 + r; i < rows * (D / 8); i += 256) out[i] = make_uint4(0, 0, 0, 0);
+    if (a.lse && hf == 0 && r < rows) a.lse[row0 + r] = -INFINITY;
   };
   int g = 0, tc = 0, e = 0;
   for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {

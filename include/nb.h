@@ -175,6 +175,35 @@ NB_API nb_status nb_attn_bwd_noalloc(const void* q, const void* k, const void* v
 NB_API nb_status nb_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
                            int k, void* stream);
 
+/*
+ * nb_tokenize_batch - a batch of DNA sequences straight to model input IDs,
+ * padded to a common length that is a multiple of 32.
+ * (NucleoByte page, section 2 items 1-2 "Fused 2-Bit Tokenization" and
+ * "Dynamic Ceiling Hardware Alignment"; section 5 "Architecture Size": a
+ * 4096-entry 6-mer vocabulary plus padding/mask, and "Evaluation Output
+ * Verification"; section 6: vocab_size 4100, input IDs drawn from 1 upward.)
+ * Model IDs, for window size k:
+ *   NB_PAD_ID (0)          padding past a sequence's last window;
+ *   raw + 1 in [1, 4^k]    a window of valid bases (raw = the nb_tokenize_kmer ID);
+ *   4^k + 1                a window holding an invalid byte;
+ *   4^k + 2                the mask ID (never written here; for the caller's masking).
+ * For k = 6 this is the page's vocabulary of 4100 (IDs 0..4099, 4099 unused).
+ * seqs      in : the batch's bases, concatenated (any alignment).
+ * offsets   in : int64 [batch + 1]: sequence b is seqs[offsets[b] .. offsets[b+1]).
+ *                Offsets that decrease give an empty sequence.
+ * input_ids out: int64 [batch][n_pad], 16-byte aligned.  Row b holds the model
+ *                IDs of its windows (stride 1) followed by NB_PAD_ID.
+ * lengths   out: int32 [batch] or NULL: the number of windows of each sequence,
+ *                max(0, bases - k + 1), the attention's per-sequence length.
+ * n_pad: a multiple of 32 (the dynamic ceiling: the smallest multiple of 32 that
+ *        holds the longest sequence's windows); a sequence with more windows
+ *        keeps its first n_pad and reports lengths[b] = n_pad.
+ * k: 1..7.  batch >= 0.
+ */
+#define NB_PAD_ID 0
+NB_API nb_status nb_tokenize_batch(const uint8_t* seqs, const int64_t* offsets, int batch, int k,
+                                   int64_t* input_ids, int32_t* lengths, int n_pad, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,6 +18,15 @@ Definition written out here:
 * The packed base stream holds 4 bases per byte, the first base in bits 7..6;
   an invalid base is stored as 0 (a 2-bit code cannot hold it; the ID stream
   carries the flag); unused slots of the final byte are 0.
+
+Model input IDs of a batch (section 2 item 2 "Dynamic Ceiling Hardware
+Alignment": a batch is padded up to the nearest multiple of the block size 32;
+section 5: a 4096-entry vocabulary "plus padding/mask"; section 6: vocab_size
+4100 and input IDs drawn from 1 upward).  Reading: ID 0 is padding and every
+raw window ID is shifted up by one, so a window of valid bases has ID raw + 1
+in 1..4**k, a window with an invalid byte 4**k + 1, and the mask ID is
+4**k + 2.  The page's MLM example supports the shift: its masked position 12
+holds the window TGGGAA (raw 3744) and the page prints ID 3745 there.
 """
 
 from __future__ import annotations
@@ -67,3 +76,31 @@ def pack_2bit(seq) -> np.ndarray:
     quads = padded.reshape(nbytes, 4)
     out = (quads[:, 0] << 6) | (quads[:, 1] << 4) | (quads[:, 2] << 2) | quads[:, 3]
     return out.astype(np.uint8)
+
+
+PAD_ID = 0
+
+
+def ceiling(n_windows_max: int, block: int = 32) -> int:
+    """The dynamic ceiling: the smallest multiple of `block` holding n_windows_max."""
+    return -(-max(int(n_windows_max), 0) // block) * block
+
+
+def model_ids_batch(seqs, k: int = 6, n_pad: int | None = None):
+    """Model input IDs (int64 [batch, n_pad]) and window counts (int32 [batch]).
+
+    Row b holds kmer_ids(seqs[b]) + 1 (the flag window becomes 4**k + 1), then
+    PAD_ID; n_pad defaults to the ceiling of the longest row.  Rows longer than
+    n_pad keep their first n_pad windows.
+    """
+    raw = [kmer_ids(s, k) for s in seqs]
+    counts = [r.shape[0] for r in raw]
+    if n_pad is None:
+        n_pad = ceiling(max(counts, default=0))
+    ids = np.full((len(seqs), n_pad), PAD_ID, dtype=np.int64)
+    lengths = np.zeros(len(seqs), dtype=np.int32)
+    for b, r in enumerate(raw):
+        m = min(r.shape[0], n_pad)
+        ids[b, :m] = r[:m].astype(np.int64) + 1
+        lengths[b] = m
+    return ids, lengths

@@ -108,3 +108,22 @@ def test_tokenizer_mutation_is_caught(name, old, new):
     ok &= mod.kmer_ids(b"ACGTNA", 6).tolist() == [4096]
     ok &= mod.pack_2bit(b"ACGTG").tolist() == [0x1B, 0x80]
     assert not ok, name
+
+
+MODEL_ID_MUTATIONS = [
+    ("no id shift", "ids[b, :m] = r[:m].astype(np.int64) + 1", "ids[b, :m] = r[:m].astype(np.int64)"),
+    ("pad id", "PAD_ID = 0", "PAD_ID = 4099"),
+    ("ceiling rounds down", "return -(-max(int(n_windows_max), 0) // block) * block",
+     "return (max(int(n_windows_max), 0) // block) * block"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MODEL_ID_MUTATIONS, ids=[m[0] for m in MODEL_ID_MUTATIONS])
+def test_model_id_mutation_is_caught(name, old, new):
+    assert old in SRC_TOK, name
+    mod = _load_mutant(SRC_TOK.replace(old, new), "mutant_tok_ids")
+    page_seq = b"CCCAGGGTCCGATGGGAAAGTGTAGCCTGC"
+    ids, lengths = mod.model_ids_batch([page_seq, b"ACG"], 6)
+    ok = ids.shape == (2, 32) and int(ids[0, 12]) == 3745 and lengths.tolist() == [25, 0]
+    ok = ok and ids[0, 25:].tolist() == [0] * 7 and ids[1].tolist() == [0] * 32
+    assert not ok, name

@@ -101,3 +101,49 @@ def test_pack_random_matches_bitstring_parse():
         bits += "0" * (-len(bits) % 8)
         want = [int(bits[i:i + 8], 2) for i in range(0, len(bits), 8)]
         assert pack_2bit(s.encode()).tolist() == want
+
+
+# ---------------------------------------------------------------- model IDs
+
+def test_model_ids_reproduce_the_page_masked_position():
+    """With padding at 0 and window IDs shifted up by one, the model ID at the
+    page's masked position 12 is the ID the page prints there (3745)."""
+    from oracle.tokenizer import model_ids_batch
+
+    seq, idx, kmers = _golden_example()
+    ids, lengths = model_ids_batch([seq.encode()], 6)
+    assert int(ids[0, idx]) == kmers[0][1] == 3745
+    # every window: its base-4 value plus one; then padding up to the ceiling 32
+    assert lengths.tolist() == [25] and ids.shape == (1, 32)
+    for p in range(25):
+        assert int(ids[0, p]) == int(seq[p:p + 6].translate(BASE4), 4) + 1
+    assert ids[0, 25:].tolist() == [0] * 7
+
+
+def test_model_ids_flag_pad_and_vocabulary():
+    from oracle.tokenizer import model_ids_batch
+
+    ids, lengths = model_ids_batch([b"ACGTNACGTAC", b"ACGTA", b"", b"TTTTTTT"], 6)
+    assert lengths.tolist() == [6, 0, 0, 2]
+    assert ids.shape == (4, 32)
+    # windows 0..5 of ACGTNACGTAC: those holding the N (byte 4) are 4^6 + 1
+    assert ids[0, :6].tolist() == [4097] * 5 + [int("ACGTAC".translate(BASE4), 4) + 1]
+    assert ids[3, :2].tolist() == [4096, 4096]  # TTTTTT = 4095 raw
+    assert ids[1].tolist() == [0] * 32 and ids[2].tolist() == [0] * 32
+    assert int(ids.max()) < 4100  # the page's vocab_size
+
+
+@pytest.mark.parametrize("windows,ceiling", [(0, 0), (1, 32), (31, 32), (32, 32), (33, 64),
+                                             (4091, 4096), (4096, 4096)])
+def test_dynamic_ceiling(windows, ceiling):
+    from oracle.tokenizer import ceiling as ceil32
+
+    assert ceil32(windows) == ceiling
+
+
+def test_model_ids_truncate_to_explicit_pad():
+    from oracle.tokenizer import model_ids_batch
+
+    ids, lengths = model_ids_batch([b"ACGTACGTACGT"], 3, n_pad=4)
+    assert lengths.tolist() == [4]
+    assert ids[0].tolist() == [int(w.translate(BASE4), 4) + 1 for w in ("ACG", "CGT", "GTA", "TAC")]

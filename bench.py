@@ -320,6 +320,72 @@ def run_tokenizer_workload(args):
     print(json.dumps(line), flush=True)
 
 
+def run_batch_ids_workload(args):
+    """The batch-to-model-IDs tokenizer alone (one GPU): windows/s and the
+    fraction of the HBM roofline (bases and offsets read, padded int64 IDs and
+    lengths written)."""
+    import numpy as np
+    import torch
+
+    import block_sparse_local_nb_b200 as nb
+    from block_sparse_local_nb_b200.inputs import make_dna_batch
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    blob, offsets = make_dna_batch()
+    batch = offsets.size - 1
+    windows = np.maximum(np.diff(offsets) - 5, 0)
+    n_pad = int(-(-windows.max() // 32) * 32)
+    seqs = torch.from_numpy(blob).to(dev)
+    off = torch.from_numpy(offsets).to(dev)
+    ids = torch.empty((batch, n_pad), dtype=torch.int64, device=dev)
+    lengths = torch.empty(batch, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sptr = stream.cuda_stream
+    for _ in range(args.warmup):
+        nb.nb_tokenize_batch(seqs, off, batch, 6, ids, lengths, n_pad, sptr)
+    torch.cuda.synchronize(dev)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(0)
+    with sampler:
+        start.record(stream)
+        for _ in range(args.steps):
+            nb.nb_tokenize_batch(seqs, off, batch, 6, ids, lengths, n_pad, sptr)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(end) / args.steps
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    alg_bytes = blob.size + 8 * offsets.size + 8 * batch * n_pad + 4 * batch
+    achieved = alg_bytes / (ms / 1e3) / 1e9
+    line = {
+        "metric": "batch tokenizer to model IDs windows/s and % of HBM roofline",
+        "value": float(windows.sum()) / (ms / 1e3), "unit": "windows/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+        "config": {"workload": "dna_batch_ids", "sequences": int(batch), "bases": int(blob.size),
+                   "n_pad": n_pad, "k": 6, "n_fraction": 0.01,
+                   "l2": f"output ({8 * batch * n_pad / 2**20:.0f} MiB) larger than the 126 MB L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm,
+                     "traffic": recorded_traffic("tokenize_batch_kernel", "dna_batch_ids"),
+                     "kernel": "tokenize_batch_kernel", "peak_source": peak_kind},
+        "gpu_launches": args.steps, "clocks": sampler.summary(),
+    }
+    if not args.no_cpu_baseline:
+        from oracle.tokenizer import model_ids_batch
+
+        sample = [blob[offsets[i]:offsets[i + 1]].tobytes() for i in range(256)]
+        t0 = time.perf_counter()
+        model_ids_batch(sample, 6, n_pad=n_pad)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": float(windows[:256].sum()) / dt, "unit": "windows/s",
+                                "cores": 1, "kind": "oracle",
+                                "sample": "first 256 sequences through the NumPy oracle"}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -340,6 +406,10 @@ def main():
     if args.workload == "dna_2p28":
         if args.impl == "native" and int(os.environ.get("RANK", "0")) == 0:
             run_tokenizer_workload(args)
+        return
+    if args.workload == "dna_batch_ids":
+        if args.impl == "native" and int(os.environ.get("RANK", "0")) == 0:
+            run_batch_ids_workload(args)
         return
     w = WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", "0"))

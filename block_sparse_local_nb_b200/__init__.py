@@ -16,5 +16,6 @@ from .binding import (  # noqa: F401
     nb_attn_fwd,
     nb_kernel_error,
     nb_status_string,
+    nb_tokenize_batch,
     nb_tokenize_kmer,
 )

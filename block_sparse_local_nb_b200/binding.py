@@ -31,6 +31,7 @@ _SIGS = [
     ("nb_attn_bwd", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                          _I, _I, _I, _I, _I, _I, _P]),
     ("nb_tokenize_kmer", _I, [_P, ctypes.c_int64, _P, _P, _I, _P]),
+    ("nb_tokenize_batch", _I, [_P, _P, _I, _I, _P, _P, _I, _P]),
 ]
 
 
@@ -119,4 +120,12 @@ def nb_tokenize_kmer(seq, length, ids, packed, k=6, stream=None, check=True):
     st = lib().nb_tokenize_kmer(_ptr(seq), length, _ptr(ids), _ptr(packed), k, _stream(stream))
     if check:
         _check(st, "nb_tokenize_kmer")
+    return st
+
+
+def nb_tokenize_batch(seqs, offsets, batch, k, input_ids, lengths, n_pad, stream=None, check=True):
+    st = lib().nb_tokenize_batch(_ptr(seqs), _ptr(offsets), batch, k, _ptr(input_ids),
+                                 _ptr(lengths), n_pad, _stream(stream))
+    if check:
+        _check(st, "nb_tokenize_batch")
     return st

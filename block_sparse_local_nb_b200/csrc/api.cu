@@ -180,4 +180,21 @@ nb_status nb_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8
   return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
 }
 
+nb_status nb_tokenize_batch(const uint8_t* seqs, const int64_t* offsets, int batch, int k,
+                            int64_t* input_ids, int32_t* lengths, int n_pad, void* stream) {
+  if (batch < 0 || n_pad < 0 || n_pad % NB_BLOCK != 0) return NB_ERR_INVALID_ARG;
+  if (k < 1 || k > 7 || batch > 65535) return NB_ERR_UNSUPPORTED;
+  if (batch == 0) return NB_OK;
+  if (!seqs || !offsets || (n_pad > 0 && !input_ids)) return NB_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(input_ids) & 15u) || (reinterpret_cast<uintptr_t>(offsets) & 7u) ||
+      (reinterpret_cast<uintptr_t>(lengths) & 3u))
+    return NB_ERR_MISALIGNED;
+  if (n_pad == 0 && !lengths) return NB_OK;
+  nb_status st = check_device();
+  if (st != NB_OK) return st;
+  cudaError_t e = nb::launch_tokenize_batch(seqs, offsets, batch, k, input_ids, lengths, n_pad,
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
+}
+
 }  // extern "C"

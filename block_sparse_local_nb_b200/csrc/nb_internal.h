@@ -86,6 +86,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 cudaError_t launch_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
                                  int k, cudaStream_t stream);
+cudaError_t launch_tokenize_batch(const uint8_t* seqs, const int64_t* offsets, int batch, int k,
+                                  int64_t* ids, int32_t* lengths, int n_pad, cudaStream_t stream);
 cudaError_t launch_attn_fwd_f32(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_bwd_bf16(const AttnArgs& a, cudaStream_t stream);

@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(256) tokenize_kmer_kernel(const uint8_t* __res
                                                             uint8_t* __restrict__ packed,
                                                             int64_t nchunks, bool ids_vec,
                                                             bool packed_vec) {
+  __shared__ uint4 stage[256 * 4];
   pdl_trigger();
   pdl_wait();
   const int64_t nwin = len - K + 1;  // number of windows (may be <= 0)
@@ -104,7 +105,30 @@ __global__ void __launch_bounds__(256) tokenize_kmer_kernel(const uint8_t* __res
 #pragma unroll
     for (int i = 0; i < 10; ++i) wd[i] = classify(w[i]);
 
-    if (ids != nullptr) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wbase = base - lane * kBases;  // the warp's first window
+    if (ids != nullptr && ids_vec && wbase + 32 * kBases <= nwin) {
+      // whole warp in range: stage the 64-byte ID runs (16-byte chunks swizzled),
+      // then write the warp's 2 KB span with coalesced 512-byte stores
+      uint4* mine = stage + threadIdx.x * 4;
+      const int sw = (lane >> 1) & 3;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t out[8];
+        window_ids<K>(wd, h, out);
+        mine[(2 * h) ^ sw] = make_uint4(out[0], out[1], out[2], out[3]);
+        mine[(2 * h + 1) ^ sw] = make_uint4(out[4], out[5], out[6], out[7]);
+      }
+      __syncwarp();
+      const uint4* wstage = stage + (threadIdx.x - lane) * 4;
+      uint4* dst = reinterpret_cast<uint4*>(ids + wbase);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int c = 32 * r + lane, from = c >> 2;
+        __stcs(dst + c, wstage[from * 4 + ((c & 3) ^ ((from >> 1) & 3))]);
+      }
+      __syncwarp();  // the staging is rewritten by the next iteration
+    } else if (ids != nullptr) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t out[8];
@@ -149,7 +173,97 @@ cudaError_t launch_k(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* pa
                     ids, packed, nchunks, ids_vec, packed_vec);
 }
 
+// Batch to model input IDs: thread = 32 consecutive windows of one sequence
+// (blockIdx.y).  Model ID = raw window ID + 1, so the flag 4^K becomes 4^K + 1;
+// windows at or past the sequence's window count (or n_pad) are padding (0).
+template <int K>
+__global__ void __launch_bounds__(128) tokenize_batch_kernel(const uint8_t* __restrict__ seqs,
+                                                             const int64_t* __restrict__ offsets,
+                                                             int64_t* __restrict__ ids,
+                                                             int32_t* __restrict__ lengths,
+                                                             int n_pad) {
+  // per thread: its 32 IDs (256 bytes) staged with a 16-byte-chunk swizzle, then
+  // each warp writes its contiguous 8 KB span with 512-byte coalesced stores
+  __shared__ uint4 stage[128 * 16];
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t s0 = offsets[b];
+  const int64_t nbases = max(offsets[b + 1] - s0, (int64_t)0);
+  const int len = static_cast<int>(min(max(nbases - K + 1, (int64_t)0), (int64_t)n_pad));
+  if (lengths != nullptr && blockIdx.x == 0 && threadIdx.x == 0) lengths[b] = len;
+  const int t0 = (blockIdx.x * blockDim.x + threadIdx.x) * kBases;  // first window
+  uint4* mine = stage + threadIdx.x * 16;
+  if (t0 < n_pad && t0 >= len) {  // all padding
+#pragma unroll
+    for (int j = 0; j < 16; ++j) mine[j ^ (lane & 15)] = make_uint4(0, 0, 0, 0);
+  } else if (t0 < n_pad) {
+    // bases t0 .. t0 + 39 of this sequence (past its end: 0, an invalid byte)
+    const uint8_t* src = seqs + s0 + t0;
+    const int64_t avail = nbases - t0;
+    uint32_t w[10];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const int p = 4 * i + bb;
+        const uint32_t byte = p < avail ? __ldg(src + p) : 0u;
+        x |= byte << (8 * bb);
+      }
+      w[i] = x;
+    }
+    Word wd[10];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) wd[i] = classify(w[i]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t out[8];
+      window_ids<K>(wd, h, out);
+#pragma unroll
+      for (int j = 0; j < 16; j += 2) {
+        const int t = t0 + 16 * h + j;
+        const uint32_t r0 = out[j >> 1] & 0xFFFFu, r1 = out[j >> 1] >> 16;
+        const uint32_t m0 = t < len ? r0 + 1u : 0u, m1 = t + 1 < len ? r1 + 1u : 0u;
+        mine[(8 * h + (j >> 1)) ^ (lane & 15)] = make_uint4(m0, 0u, m1, 0u);
+      }
+    }
+  }
+  __syncwarp();
+  const int wt0 = t0 - lane * kBases;  // the warp's first window
+  const int count = min(32 * kBases, n_pad - wt0) / 2;  // 16-byte chunks of the warp's span
+  uint4* dst = reinterpret_cast<uint4*>(ids + static_cast<int64_t>(b) * n_pad + wt0);
+  const uint4* wstage = stage + warp * 32 * 16;
+  for (int c = lane; c < count; c += 32) {
+    const int from = c >> 4;  // the lane that produced chunk c
+    __stcs(dst + c, wstage[from * 16 + ((c & 15) ^ (from & 15))]);
+  }
+}
+
+template <int K>
+cudaError_t launch_batch_k(const uint8_t* seqs, const int64_t* offsets, int batch, int64_t* ids,
+                           int32_t* lengths, int n_pad, cudaStream_t stream) {
+  const int chunks = n_pad / kBases;
+  const unsigned gx = static_cast<unsigned>(chunks > 0 ? (chunks + 127) / 128 : 1);
+  return launch_pdl(tokenize_batch_kernel<K>, dim3(gx, static_cast<unsigned>(batch)), dim3(128), 0,
+                    stream, seqs, offsets, ids, lengths, n_pad);
+}
+
 }  // namespace
+
+cudaError_t launch_tokenize_batch(const uint8_t* seqs, const int64_t* offsets, int batch, int k,
+                                  int64_t* ids, int32_t* lengths, int n_pad, cudaStream_t stream) {
+  switch (k) {
+    case 1: return launch_batch_k<1>(seqs, offsets, batch, ids, lengths, n_pad, stream);
+    case 2: return launch_batch_k<2>(seqs, offsets, batch, ids, lengths, n_pad, stream);
+    case 3: return launch_batch_k<3>(seqs, offsets, batch, ids, lengths, n_pad, stream);
+    case 4: return launch_batch_k<4>(seqs, offsets, batch, ids, lengths, n_pad, stream);
+    case 5: return launch_batch_k<5>(seqs, offsets, batch, ids, lengths, n_pad, stream);
+    case 6: return launch_batch_k<6>(seqs, offsets, batch, ids, lengths, n_pad, stream);
+    default: return launch_batch_k<7>(seqs, offsets, batch, ids, lengths, n_pad, stream);
+  }
+}
 
 cudaError_t launch_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
                                  int k, cudaStream_t stream) {

@@ -119,3 +119,21 @@ def make_dna(nbytes: int = DNA_BYTES, seed: int = DNA_SEED, n_prob: float = DNA_
     out = letters[u & 3]
     out[u < int(round(n_prob * denom))] = ord("N")
     return out
+
+
+# batch of DNA sequences for the model-ID tokenizer: 8192 sequences whose base
+# counts are uniform in [1024, 4101] (so the padded width is 4096 windows),
+# bases as in make_dna
+DNA_BATCH = 8192
+DNA_BATCH_BASES = (1024, 4101)
+DNA_BATCH_SEED = 6
+
+
+def make_dna_batch(count: int = DNA_BATCH, bases=DNA_BATCH_BASES, seed: int = DNA_BATCH_SEED):
+    """(blob uint8, offsets int64 [count + 1]): the sequences concatenated."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(bases[0], bases[1] + 1, size=count).astype(np.int64)
+    offsets = np.zeros(count + 1, dtype=np.int64)
+    np.cumsum(lens, out=offsets[1:])
+    blob = make_dna(int(offsets[-1]), seed=seed + 1000)
+    return blob, offsets

@@ -135,3 +135,26 @@ def test_bwd_rejects_invalid_arguments(lib, kw, status):
 def test_tokenize_rejects_invalid_arguments(lib, args, status):
     seq, n, ids, packed, k = args
     assert lib.nb_tokenize_kmer(seq, n, ids, packed, k, None) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=-1), NB_ERR_INVALID_ARG),
+    (dict(n_pad=48), NB_ERR_INVALID_ARG),       # not a multiple of 32
+    (dict(n_pad=-32), NB_ERR_INVALID_ARG),
+    (dict(k=0), NB_ERR_UNSUPPORTED),
+    (dict(k=8), NB_ERR_UNSUPPORTED),
+    (dict(batch=70000), NB_ERR_UNSUPPORTED),
+    (dict(seqs=None), NB_ERR_INVALID_ARG),
+    (dict(offsets=None), NB_ERR_INVALID_ARG),
+    (dict(ids=None), NB_ERR_INVALID_ARG),
+    (dict(ids=40), NB_ERR_MISALIGNED),
+    (dict(offsets=12), NB_ERR_MISALIGNED),
+    (dict(lengths=18), NB_ERR_MISALIGNED),
+    (dict(batch=0), NB_OK),
+    (dict(n_pad=0, lengths=None), NB_OK),
+])
+def test_tokenize_batch_rejects_invalid_arguments(lib, kw, status):
+    args = dict(seqs=16, offsets=16, batch=2, k=6, ids=16, lengths=16, n_pad=64)
+    args.update(kw)
+    assert lib.nb_tokenize_batch(args["seqs"], args["offsets"], args["batch"], args["k"], args["ids"],
+                                 args["lengths"], args["n_pad"], None) == status

@@ -100,3 +100,79 @@ def test_full_size_2p28_bit_exact():
     got_ids = ids.cpu().numpy().view(np.uint16)
     np.testing.assert_array_equal(got_ids, kmer_ids(s, 6))
     np.testing.assert_array_equal(packed.cpu().numpy(), pack_2bit(s))
+
+
+# ------------------------------------------------------- batch to model IDs
+
+def _run_batch(seqs, k=6, n_pad=None, lead=3):
+    """nb_tokenize_batch on `seqs` concatenated after `lead` bytes (so sequences
+    start at arbitrary byte offsets); returns (ids, lengths) and checks that the
+    guard row after the output and the guard entry after the lengths are untouched."""
+    from oracle.tokenizer import ceiling
+
+    offsets = [lead]
+    for s in seqs:
+        offsets.append(offsets[-1] + len(s))
+    # bases before the first and after the last sequence must not be read into them
+    blob = b"ACGT" * 4 + b"Z" * lead + b"".join(seqs) + b"ACGT" * 4
+    offsets = [o + 16 for o in offsets]
+    dev = torch.frombuffer(bytearray(blob), dtype=torch.uint8).cuda()
+    off = torch.tensor(offsets, dtype=torch.int64, device="cuda")
+    if n_pad is None:
+        n_pad = ceiling(max([max(len(s) - k + 1, 0) for s in seqs], default=0))
+    ids = torch.full((len(seqs) + 1, max(n_pad, 1)), -7, dtype=torch.int64, device="cuda")
+    lengths = torch.full((len(seqs) + 1,), -7, dtype=torch.int32, device="cuda")
+    nb.nb_tokenize_batch(dev, off, len(seqs), k, ids, lengths, n_pad)
+    torch.cuda.synchronize()
+    assert (ids[len(seqs)] == -7).all() and int(lengths[len(seqs)]) == -7
+    return ids[:len(seqs), :n_pad].cpu().numpy(), lengths[:len(seqs)].cpu().numpy()
+
+
+def test_batch_page_example():
+    from oracle.tokenizer import model_ids_batch
+
+    seq = [p for p in read_golden("nucleobyte_mlm_example.txt") if p[0] == "sequence"][0][1]
+    ids, lengths = _run_batch([seq.encode()])
+    want, want_len = model_ids_batch([seq.encode()], 6)
+    assert np.array_equal(ids, want) and np.array_equal(lengths, want_len)
+    assert int(ids[0, 12]) == 3745
+
+
+@pytest.mark.parametrize("k", [1, 3, 6, 7])
+def test_batch_random_matches_oracle(k):
+    from oracle.tokenizer import model_ids_batch
+
+    rng = np.random.default_rng(40 + k)
+    alphabet = np.frombuffer(b"ACGTACGTACGTNacgt\n", dtype=np.uint8)
+    lens = [0, 1, k - 1, k, k + 1, 31 + k, 32 + k, 33 + k] + rng.integers(0, 3000, 40).tolist()
+    seqs = [alphabet[rng.integers(0, alphabet.size, int(n))].tobytes() for n in lens]
+    ids, lengths = _run_batch(seqs, k, lead=k)
+    want, want_len = model_ids_batch(seqs, k)
+    assert np.array_equal(lengths, want_len)
+    assert np.array_equal(ids, want)
+
+
+def test_batch_truncates_to_n_pad():
+    from oracle.tokenizer import model_ids_batch
+
+    rng = np.random.default_rng(3)
+    seqs = [rng.choice(np.frombuffer(b"ACGT", np.uint8), n).tobytes() for n in (10, 100, 300)]
+    ids, lengths = _run_batch(seqs, 6, n_pad=64)
+    want, want_len = model_ids_batch(seqs, 6, n_pad=64)
+    assert lengths.tolist() == [5, 64, 64] == want_len.tolist()
+    assert np.array_equal(ids, want)
+
+
+def test_batch_training_sized():
+    """1024 sequences of up to 4101 bases (the training batches' shape)."""
+    from oracle.tokenizer import model_ids_batch
+
+    rng = np.random.default_rng(11)
+    alphabet = np.frombuffer(b"ACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTACGTN",
+                             np.uint8)
+    seqs = [alphabet[rng.integers(0, alphabet.size, int(n))].tobytes()
+            for n in rng.integers(1024, 4102, 1024)]
+    ids, lengths = _run_batch(seqs, 6)
+    want, want_len = model_ids_batch(seqs, 6)
+    assert ids.shape == (1024, 4096)
+    assert np.array_equal(lengths, want_len) and np.array_equal(ids, want)

@@ -271,7 +271,10 @@ cudaError_t launch_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids,
   if (nchunks == 0 || (ids == nullptr && packed == nullptr)) return cudaSuccess;
   const int threads = 256;
   int64_t blocks = (nchunks + threads - 1) / threads;
-  if (blocks > (1 << 30)) blocks = 1 << 30;  // grid-stride loop covers the rest
+  // a few waves of blocks that loop over the rest (measured: fewer, longer-lived
+  // blocks beat one short block per 8 KB of input)
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
+  if (blocks > cap) blocks = cap;
   const bool aligned = (reinterpret_cast<uintptr_t>(seq) & 15u) == 0;
   const bool ids_vec = (reinterpret_cast<uintptr_t>(ids) & 15u) == 0;
   const bool packed_vec = (reinterpret_cast<uintptr_t>(packed) & 7u) == 0;

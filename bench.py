@@ -158,7 +158,7 @@ def algorithmic(w, lengths):
     return {
         "tokens": tok,
         "fwd_bytes": th * (4 * w.d * e + 4),   # read Q K V, write O and lse
-        "bwd_bytes": th * (8 * w.d * e + 4),   # read Q K V O dO lse, write dQ dK dV
+        "bwd_bytes": th * (8 * w.d * e + 8),   # read Q K V O dO, write dQ dK dV; row term D
         "fwd_flops": 4 * w.d * pairs,          # Q K^T and P V
         "bwd_flops": 10 * w.d * pairs,         # S, dP, dV, dK, dQ
         "pairs": pairs,

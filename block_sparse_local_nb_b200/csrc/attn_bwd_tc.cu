@@ -48,11 +48,11 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int D>
 struct Cfg {
   // D = 64: K/V tiles double-buffered, three Q/dO stages; P^T kept in TMEM
-  // (64 spare columns) as the A operand of dV, which leaves room for a dQ
-  // staging buffer of its own.
+  // (64 spare columns) as the A operand of dV.
   // D = 128: TMEM is full (dQ reuses the S columns, so S/dP of chunk G + 1
-  // waits until dQ of chunk G is read out), P^T goes through shared memory
-  // and dQ is staged in the chunk's Q/dO buffer.
+  // waits until dQ of chunk G is read out) and P^T goes through shared memory.
+  // Both stage dQ through one 128 x 32 fp32 box, so a chunk's Q/dO buffer is
+  // free as soon as its gradient products complete.
   static constexpr bool kPTmem = D == 64;
   static constexpr int NKV = D == 64 ? 2 : 1;  // K/V tile buffers
   static constexpr int NS = D == 64 ? 3 : 1;   // Q/dO chunk stages
@@ -62,11 +62,11 @@ struct Cfg {
   static constexpr int oQ = NKV * 2 * kTile;     // stage s: Q at oQ + 2 s kTile, dO after it
   static constexpr int oP = oQ + NS * 2 * kTile;  // P^T tile (shared-memory variant only)
   static constexpr int oDS = oP + (kPTmem ? 0 : kPT);
-  static constexpr int oStg = oDS + kPT;  // dQ staging box (TMEM-P variant only)
+  static constexpr int oStg = oDS + kPT;  // dQ staging box (one 128 x 32 fp32 box)
   // The dK/dV epilogue of an item is deferred past the next item's first
   // chunk when the next item's K/V tile has a buffer of its own (D = 64).
   static constexpr bool kDefer = NKV > 1;
-  static constexpr int oLD = oStg + (kPTmem ? kSlab : 0);  // stage s: -lse log2e, D
+  static constexpr int oLD = oStg + kSlab;  // stage s: -lse log2e, D
   static constexpr int oBar = oLD + NS * 1024;
   static constexpr int bKVFull = 0, bKVFree = bKVFull + NKV, bQDFull = bKVFree + NKV,
                        bQDFree = bQDFull + NS, bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1,
@@ -269,7 +269,7 @@ __device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uin
       }
       mma_commit(bar + 8 * C::bPDSFree);
       mma_commit(bar + 8 * C::bDQFull);
-      if (C::kPTmem) mma_commit(bar + 8 * (C::bQDFree + st));  // Q/dO of the chunk consumed
+      mma_commit(bar + 8 * (C::bQDFree + st));  // Q/dO of the chunk consumed
       if (c == x.nch - 1) mma_commit(bar + 8 * C::bDKVFull);
     }
     g += x.nch;
@@ -506,30 +506,34 @@ __device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint8_
     if (x.nch == 0) continue;
     const int bh = x.b * a.heads + x.h;
     for (int c = 0; c < x.nch; ++c) {
-      const int G = g + c, st = G % C::NS;
+      const int G = g + c;
       const int q0 = (x.I0 + 4 * c) * kBlock;
       if (!all_ok(mbar_wait(bar + 8 * C::bDQFull, G & 1))) return kErrDQFull;
       tc_fence_after();
-      if constexpr (C::kPTmem) {
-        // whole dQ_c row in registers, then one 32-column box per pass through the
-        // staging buffer
-        float v[D / 32][32];
+      // dQ_c through the staging box, one 32-column box per pass; the row is read
+      // from TMEM 64 columns at a time and its TMEM released after the last read
+      uint8_t* stg = gbase + C::oStg;
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) tmem_ld32(trow + C::tDQ + 32 * j, v[j]);
+      for (int grp = 0; grp < D / 64; ++grp) {
+        float v[2][32];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) tmem_ld32(trow + C::tDQ + 64 * grp + 32 * jj, v[jj]);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) reg_fence(v[j]);
-        tc_fence_before();
-        mbar_arrive(bar + 8 * C::bDQFree);
-        uint8_t* stg = gbase + C::oStg;
+        for (int jj = 0; jj < 2; ++jj) reg_fence(v[jj]);
+        if (grp == D / 64 - 1) {
+          tc_fence_before();
+          mbar_arrive(bar + 8 * C::bDQFree);
+        }
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * grp + jj;      // box (32 columns) within the row
           const int k = G * (D / 32) + j;  // global pass index
           if (!all_ok(mbar_wait(bar + 8 * C::bStgFree, (k & 1) ^ 1))) return kErrStgFree;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             *reinterpret_cast<float4*>(stg + r * 128 + ((u ^ (r & 7)) << 4)) =
-                make_float4(v[j][4 * u], v[j][4 * u + 1], v[j][4 * u + 2], v[j][4 * u + 3]);
+                make_float4(v[jj][4 * u], v[jj][4 * u + 1], v[jj][4 * u + 2], v[jj][4 * u + 3]);
           fence_proxy_async_smem();
           mbar_arrive(bar + 8 * C::bStg);  // this thread's row of the box is written
           if (leader) {
@@ -539,33 +543,6 @@ __device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint8_
             bulk_wait_read0();
             mbar_arrive(bar + 8 * C::bStgFree);
           }
-        }
-      } else {
-        // all D/32 boxes at once in the chunk's Q/dO buffer (free once dQ_c is done)
-        uint8_t* stg = gbase + C::oQ + st * 2 * C::kTile;
-#pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
-          float v[32];
-          tmem_ld32(trow + C::tDQ + 32 * j, v);
-          tmem_wait_ld();
-          reg_fence(v);
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<float4*>(stg + j * kSlab + r * 128 + ((u ^ (r & 7)) << 4)) =
-                make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-        }
-        tc_fence_before();
-        mbar_arrive(bar + 8 * C::bDQFree);
-        fence_proxy_async_smem();
-        mbar_arrive(bar + 8 * C::bStg);
-        if (leader) {
-          if (!mbar_wait(bar + 8 * C::bStg, G & 1)) return kErrStg;
-#pragma unroll
-          for (int j = 0; j < D / 32; ++j)
-            tma_reduce_add_3d(tdq, base + C::oQ + st * 2 * C::kTile + j * kSlab, 32 * j, q0, bh);
-          bulk_commit();
-          bulk_wait_read0();
-          mbar_arrive(bar + 8 * (C::bQDFree + st));
         }
       }
     }

@@ -262,6 +262,9 @@ __device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uin
           mma_bf16_ss(tmem + C::tDV, desc_add(dP, off), desc_add(ddO, mn), kIdKV, acc || k > 0);
         mma_bf16_ss(tmem + C::tDK, desc_add(dSk, off), desc_add(dQ, mn), kIdKV, acc || k > 0);
       }
+      // Q and dO are last read by the products above: their buffer can refill
+      // while the dQ product runs
+      mma_commit(bar + 8 * (C::bQDFree + st));
 #pragma unroll
       for (int k = 0; k < kRows / 16; ++k) {  // k over the tile's keys
         const uint32_t mn = (k * 2048) >> 4;
@@ -269,7 +272,6 @@ __device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uin
       }
       mma_commit(bar + 8 * C::bPDSFree);
       mma_commit(bar + 8 * C::bDQFull);
-      mma_commit(bar + 8 * (C::bQDFree + st));  // Q/dO of the chunk consumed
       if (c == x.nch - 1) mma_commit(bar + 8 * C::bDKVFull);
     }
     g += x.nch;

@@ -29,6 +29,11 @@ Layout: every tensor is [batch, heads, n, d] (d innermost); log-sum-exp is
 [batch, heads, n].  ``lengths`` is an int array [batch] with 0 <= L <= n
 (None means every sequence is full length).
 
+Causal band (a variant the page does not print; the plainest causal reading
+of its band): query q in block i sees key k in block j only when
+i - R <= j <= i and k <= q, i.e. the band's lower half plus the token-level
+causal triangle of the diagonal block.  Every function takes ``causal``.
+
 Two restatements of the same definition are given:
 * ``*_dense``: the full n x n score matrix with the band mask applied
   (small n only);
@@ -59,15 +64,19 @@ def _lengths(lengths, batch: int, n: int) -> np.ndarray:
     return lens
 
 
-def block_band_mask(n: int, R: int, length: int | None = None, block: int = BLOCK) -> np.ndarray:
+def block_band_mask(n: int, R: int, length: int | None = None, block: int = BLOCK,
+                    causal: bool = False) -> np.ndarray:
     """Boolean visibility matrix M[q, k] for one sequence.
 
     M[q, k] is True iff the key block of k lies within R blocks of the query
-    block of q (|q // B - k // B| <= R) and k < length.  Query-row padding is
-    not part of the mask (rows q >= length are handled by the callers).
+    block of q (|q // B - k // B| <= R) and k < length; with ``causal`` also
+    k <= q.  Query-row padding is not part of the mask (rows q >= length are
+    handled by the callers).
     """
     blk = np.arange(n) // block
     m = np.abs(blk[:, None] - blk[None, :]) <= R
+    if causal:
+        m &= np.arange(n)[None, :] <= np.arange(n)[:, None]
     if length is not None:
         m &= (np.arange(n) < length)[None, :]
     return m
@@ -88,7 +97,7 @@ def _softmax_rows(S: np.ndarray):
     return P, m, l
 
 
-def attn_fwd_dense(q, k, v, R: int, lengths=None):
+def attn_fwd_dense(q, k, v, R: int, lengths=None, causal: bool = False):
     """Forward pass from the dense definition.
 
     Returns (o, lse): o [batch, heads, n, d] fp64 and lse [batch, heads, n]
@@ -103,7 +112,7 @@ def attn_fwd_dense(q, k, v, R: int, lengths=None):
     lse = np.full((batch, heads, n), -np.inf)
     for b in range(batch):
         L = int(lens[b])
-        mask = block_band_mask(n, R, L)
+        mask = block_band_mask(n, R, L, causal=causal)
         for h in range(heads):
             S = scale * (q[b, h] @ k[b, h].T)
             S = np.where(mask, S, -np.inf)
@@ -113,7 +122,7 @@ def attn_fwd_dense(q, k, v, R: int, lengths=None):
     return o, lse
 
 
-def attn_bwd_dense(q, k, v, do, R: int, lengths=None):
+def attn_bwd_dense(q, k, v, do, R: int, lengths=None, causal: bool = False):
     """Analytic gradients from the dense definition.
 
     Returns (dq, dk, dv), each [batch, heads, n, d] fp64.  P and O are
@@ -130,7 +139,7 @@ def attn_bwd_dense(q, k, v, do, R: int, lengths=None):
     dv = np.zeros_like(v)
     for b in range(batch):
         L = int(lens[b])
-        mask = block_band_mask(n, R, L)
+        mask = block_band_mask(n, R, L, causal=causal)
         for h in range(heads):
             S = np.where(mask, scale * (q[b, h] @ k[b, h].T), -np.inf)
             P = np.zeros((n, n))
@@ -147,11 +156,18 @@ def attn_bwd_dense(q, k, v, do, R: int, lengths=None):
     return dq, dk, dv
 
 
-def _band(i: int, R: int, nb: int):
-    return max(0, i - R), min(nb - 1, i + R)
+def _band(i: int, R: int, nb: int, causal: bool = False):
+    return max(0, i - R), (i if causal else min(nb - 1, i + R))
 
 
-def attn_fwd_banded(q, k, v, R: int, lengths=None):
+def _causal_cut(S: np.ndarray, r0: int, k0: int) -> np.ndarray:
+    """S with entries of keys after their query (k > q) set to -inf."""
+    qi = r0 + np.arange(S.shape[0])[:, None]
+    ki = k0 + np.arange(S.shape[1])[None, :]
+    return np.where(ki <= qi, S, -np.inf)
+
+
+def attn_fwd_banded(q, k, v, R: int, lengths=None, causal: bool = False):
     """Forward pass evaluated only on each query block's band of key blocks.
 
     Same definition and outputs as :func:`attn_fwd_dense`; memory is linear in
@@ -173,17 +189,19 @@ def attn_fwd_banded(q, k, v, R: int, lengths=None):
             rows = min(BLOCK, L - r0)
             if rows <= 0:
                 break
-            j0, j1 = _band(i, R, nb)
+            j0, j1 = _band(i, R, nb, causal)
             k0, k1 = j0 * BLOCK, min((j1 + 1) * BLOCK, L)  # keys past L are masked
             for h in range(heads):
                 S = scale * (q[b, h, r0:r0 + rows] @ k[b, h, k0:k1].T)
+                if causal:
+                    S = _causal_cut(S, r0, k0)
                 P, m, l = _softmax_rows(S)
                 o[b, h, r0:r0 + rows] = P @ v[b, h, k0:k1]
                 lse[b, h, r0:r0 + rows] = m + np.log(l)
     return o, lse
 
 
-def attn_bwd_banded(q, k, v, do, R: int, lengths=None):
+def attn_bwd_banded(q, k, v, do, R: int, lengths=None, causal: bool = False):
     """Analytic gradients evaluated only on each query block's band.
 
     Same definition and outputs as :func:`attn_bwd_dense`: for every query
@@ -208,13 +226,16 @@ def attn_bwd_banded(q, k, v, do, R: int, lengths=None):
             rows = min(BLOCK, L - r0)
             if rows <= 0:
                 break
-            j0, j1 = _band(i, R, nb)
+            j0, j1 = _band(i, R, nb, causal)
             k0, k1 = j0 * BLOCK, min((j1 + 1) * BLOCK, L)
             for h in range(heads):
                 Qi = q[b, h, r0:r0 + rows]
                 dOi = do[b, h, r0:r0 + rows]
                 Kb, Vb = k[b, h, k0:k1], v[b, h, k0:k1]
-                P, _, _ = _softmax_rows(scale * (Qi @ Kb.T))
+                S = scale * (Qi @ Kb.T)
+                if causal:
+                    S = _causal_cut(S, r0, k0)
+                P, _, _ = _softmax_rows(S)
                 Oi = P @ Vb
                 D = (dOi * Oi).sum(axis=1)
                 dP = dOi @ Vb.T

@@ -66,7 +66,7 @@ def _bwd_pin_fails(mod):
 
 
 ATT_MUTATIONS = [
-    ("band off by one", "<= R\n    if length", "< R\n    if length"),
+    ("band off by one", "blk[None, :]) <= R\n", "blk[None, :]) < R\n"),
     ("band j1 off by one", "min(nb - 1, i + R)", "min(nb - 1, i + R - 1)"),
     ("scale dropped", "scale = 1.0 / math.sqrt(d)", "scale = 1.0"),
     ("keys past length kept", "k0, k1 = j0 * BLOCK, min((j1 + 1) * BLOCK, L)  # keys past L are masked",
@@ -127,3 +127,51 @@ def test_model_id_mutation_is_caught(name, old, new):
     ok = ids.shape == (2, 32) and int(ids[0, 12]) == 3745 and lengths.tolist() == [25, 0]
     ok = ok and ids[0, 25:].tolist() == [0] * 7 and ids[1].tolist() == [0] * 32
     assert not ok, name
+
+
+def _causal_pin_fails(mod):
+    """Causal band: keys enumerated by hand per row, both oracles, fwd; and
+    central differences of the causal loss for the banded backward."""
+    rng = np.random.default_rng(5)
+    n, d, R, L = 96, 4, 1, 80
+    q, k, v, do = (rng.standard_normal((1, 1, n, d)) for _ in range(4))
+    o, _ = mod.attn_fwd_dense(q, k, v, R, lengths=[L], causal=True)
+    o_b, _ = mod.attn_fwd_banded(q, k, v, R, lengths=[L], causal=True)
+    for i in range(L):
+        keys = [j for j in range(L) if 0 <= i // 32 - j // 32 <= R and j <= i]
+        s = np.array([q[0, 0, i] @ k[0, 0, j] for j in keys]) / math.sqrt(d)
+        want = softmax(s) @ v[0, 0, keys]
+        if not (np.allclose(o[0, 0, i], want, atol=1e-10) and np.allclose(o_b[0, 0, i], want, atol=1e-10)):
+            return True
+    h = 1e-6
+
+    def loss(kk):
+        oo, _ = att.attn_fwd_dense(q, kk, v, R, lengths=[L], causal=True)  # the unmutated forward
+        return float((oo * do).sum())
+
+    _, dk, _ = mod.attn_bwd_banded(q, k, v, do, R, lengths=[L], causal=True)
+    for i in (5, 31, 32, 63, 64, 79):
+        p, m = k.copy(), k.copy()
+        p[0, 0, i, 1] += h
+        m[0, 0, i, 1] -= h
+        if abs((loss(p) - loss(m)) / (2 * h) - dk[0, 0, i, 1]) > 1e-6:
+            return True
+    return False
+
+
+CAUSAL_MUTATIONS = [
+    ("causal mask off by one", "m &= np.arange(n)[None, :] <= np.arange(n)[:, None]",
+     "m &= np.arange(n)[None, :] < np.arange(n)[:, None]"),
+    ("causal cut off by one", "return np.where(ki <= qi, S, -np.inf)", "return np.where(ki < qi, S, -np.inf)"),
+    # (keeping block i + 1 would be harmless: the triangle masks it whole)
+    ("causal band drops the diagonal block", "(i if causal else", "(i - 1 if causal else"),
+    ("causal cut skipped in backward", "                if causal:\n                    S = _causal_cut(S, r0, k0)\n                P, _, _",
+     "                P, _, _"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", CAUSAL_MUTATIONS, ids=[m[0] for m in CAUSAL_MUTATIONS])
+def test_causal_mutation_is_caught(name, old, new):
+    assert old in SRC_ATT, name
+    mod = _load_mutant(SRC_ATT.replace(old, new), "mutant_causal")
+    assert _causal_pin_fails(mod), name

@@ -174,4 +174,8 @@ CAUSAL_MUTATIONS = [
 def test_causal_mutation_is_caught(name, old, new):
     assert old in SRC_ATT, name
     mod = _load_mutant(SRC_ATT.replace(old, new), "mutant_causal")
-    assert _causal_pin_fails(mod), name
+    try:
+        caught = _causal_pin_fails(mod)
+    except ValueError:  # the mutant cannot even evaluate the pins (an empty band)
+        caught = True
+    assert caught, name

@@ -150,7 +150,11 @@ def algorithmic(w, lengths):
         tok += L
         for i in range((L + 31) // 32):
             rows = min(32, L - 32 * i)
-            lo, hi = max(0, i - w.R), min(nb_ - 1, i + w.R)
+            lo = max(0, i - w.R)
+            if getattr(w, "causal", False):  # row q sees keys lo*32 .. q
+                pairs += sum(32 * i + r - lo * 32 + 1 for r in range(rows))
+                continue
+            hi = min(nb_ - 1, i + w.R)
             keys = min((hi + 1) * 32, L) - lo * 32
             pairs += rows * keys
     th = tok * w.heads
@@ -190,8 +194,8 @@ def run_reference_arm(args, w):
         h = (step // w.batch) % w.heads
         sl = (slice(b, b + 1), slice(h, h + 1))
         Lb = [int(lengths[b])]
-        attn_fwd_banded(qn[sl], kn[sl], vn[sl], w.R, Lb)
-        attn_bwd_banded(qn[sl], kn[sl], vn[sl], don[sl], w.R, Lb)
+        attn_fwd_banded(qn[sl], kn[sl], vn[sl], w.R, Lb, causal=w.causal)
+        attn_bwd_banded(qn[sl], kn[sl], vn[sl], don[sl], w.R, Lb, causal=w.causal)
         seg = dna[b * (w.n + 5):(b + 1) * (w.n + 5)]
         kmer_ids(seg, 6)
         pack_2bit(seg)
@@ -244,8 +248,8 @@ def cpu_baseline(w):
         b, h = heads_done % w.batch, (heads_done // w.batch) % w.heads
         sl = (slice(b, b + 1), slice(h, h + 1))
         Lb = [int(lengths[b])]
-        attn_fwd_banded(qn[sl], kn[sl], vn[sl], w.R, Lb)
-        attn_bwd_banded(qn[sl], kn[sl], vn[sl], don[sl], w.R, Lb)
+        attn_fwd_banded(qn[sl], kn[sl], vn[sl], w.R, Lb, causal=w.causal)
+        attn_bwd_banded(qn[sl], kn[sl], vn[sl], don[sl], w.R, Lb, causal=w.causal)
         if h == 0:
             seg = dna[b * (w.n + 5):(b + 1) * (w.n + 5)]
             kmer_ids(seg, 6)
@@ -473,6 +477,8 @@ def main():
     torch.cuda.synchronize(dev)
 
     sptr = stream.cuda_stream
+    fwd = nb.nb_attn_fwd_causal if w.causal else nb.nb_attn_fwd
+    bwd = nb.nb_attn_bwd_causal if w.causal else nb.nb_attn_bwd
 
     def step(st, ev=None):
         if ev is not None:
@@ -480,14 +486,12 @@ def main():
         nb.nb_tokenize_kmer(st["dna"], st["dna"].numel(), st["ids"], st["packed"], 6, sptr)
         if ev is not None:
             ev[1].record(stream)
-        nb.nb_attn_fwd(st["q"], st["k"], st["v"], st["o"], st["lse"], lengths_d, B, H, N, D, R,
-                       dt_code, sptr)
+        fwd(st["q"], st["k"], st["v"], st["o"], st["lse"], lengths_d, B, H, N, D, R, dt_code, sptr)
         if ev is not None:
             ev[2].record(stream)
         if w.backward:
-            nb.nb_attn_bwd(st["q"], st["k"], st["v"], st["o"], st["do"], st["lse"], lengths_d,
-                           st["dq"], st["dk"], st["dv"], st["ws"], st["ws_bytes"], B, H, N, D, R,
-                           dt_code, sptr)
+            bwd(st["q"], st["k"], st["v"], st["o"], st["do"], st["lse"], lengths_d, st["dq"],
+                st["dk"], st["dv"], st["ws"], st["ws_bytes"], B, H, N, D, R, dt_code, sptr)
         if ev is not None:
             ev[3].record(stream)
 

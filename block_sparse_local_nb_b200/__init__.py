@@ -13,7 +13,9 @@ from .binding import (  # noqa: F401
     attn_bwd_workspace_size,
     lib,
     nb_attn_bwd,
+    nb_attn_bwd_causal,
     nb_attn_fwd,
+    nb_attn_fwd_causal,
     nb_kernel_error,
     nb_status_string,
     nb_tokenize_batch,

@@ -27,9 +27,12 @@ _SIGS = [
     ("nb_abi_version", _I, []),
     ("nb_kernel_error", _I, [ctypes.POINTER(ctypes.c_int), _I]),
     ("nb_attn_fwd", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    ("nb_attn_fwd_causal", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
     ("nb_attn_bwd_workspace_size", ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     ("nb_attn_bwd", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                          _I, _I, _I, _I, _I, _I, _P]),
+    ("nb_attn_bwd_causal", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                _I, _I, _I, _I, _I, _I, _P]),
     ("nb_tokenize_kmer", _I, [_P, ctypes.c_int64, _P, _P, _I, _P]),
     ("nb_tokenize_batch", _I, [_P, _P, _I, _I, _P, _P, _I, _P]),
 ]
@@ -102,6 +105,15 @@ def nb_attn_fwd(q, k, v, o, lse, lengths, batch, heads, n, d, R, dtype, stream=N
     return st
 
 
+def nb_attn_fwd_causal(q, k, v, o, lse, lengths, batch, heads, n, d, R, dtype, stream=None,
+                       check=True):
+    st = lib().nb_attn_fwd_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(lengths),
+                                  batch, heads, n, d, R, dtype, _stream(stream))
+    if check:
+        _check(st, "nb_attn_fwd_causal")
+    return st
+
+
 def attn_bwd_workspace_size(batch, heads, n, d, dtype) -> int:
     return int(lib().nb_attn_bwd_workspace_size(batch, heads, n, d, dtype))
 
@@ -113,6 +125,16 @@ def nb_attn_bwd(q, k, v, o, dout, lse, lengths, dq, dk, dv, workspace, workspace
                            workspace_bytes, batch, heads, n, d, R, dtype, _stream(stream))
     if check:
         _check(st, "nb_attn_bwd")
+    return st
+
+
+def nb_attn_bwd_causal(q, k, v, o, dout, lse, lengths, dq, dk, dv, workspace, workspace_bytes,
+                       batch, heads, n, d, R, dtype, stream=None, check=True):
+    st = lib().nb_attn_bwd_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                  _ptr(lengths), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                  workspace_bytes, batch, heads, n, d, R, dtype, _stream(stream))
+    if check:
+        _check(st, "nb_attn_bwd_causal")
     return st
 
 

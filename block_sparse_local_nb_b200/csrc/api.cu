@@ -70,7 +70,8 @@ nb_status check_shape(int batch, int heads, int n, int d, int R, int dtype) {
 
 nb::AttnArgs make_args(const void* q, const void* k, const void* v, const void* o,
                        const void* dout, const float* lse, const int32_t* lengths, void* dq,
-                       void* dk, void* dv, void* ws, int batch, int heads, int n, int d, int R) {
+                       void* dk, void* dv, void* ws, int batch, int heads, int n, int d, int R,
+                       bool causal) {
   nb::AttnArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout;
   a.lse = const_cast<float*>(lse);
@@ -78,8 +79,54 @@ nb::AttnArgs make_args(const void* q, const void* k, const void* v, const void* 
   a.dq = dq; a.dk = dk; a.dv = dv; a.workspace = ws;
   a.batch = batch; a.heads = heads; a.n = n; a.d = d; a.R = R;
   a.scale = static_cast<float>(1.0 / sqrt(static_cast<double>(d)));
+  a.causal = causal;
   a.err = error_word();
   return a;
+}
+
+nb_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                   const int32_t* lengths, int batch, int heads, int n, int d, int R, int dtype,
+                   void* stream, bool causal) {
+  nb_status st = check_shape(batch, heads, n, d, R, dtype);
+  if (st != NB_OK) return st;
+  if (static_cast<int64_t>(batch) * heads * n == 0) return NB_OK;
+  if (!q || !k || !v || !o) return NB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && !aligned16(lse)) || (lengths && (reinterpret_cast<uintptr_t>(lengths) & 3u)))
+    return NB_ERR_MISALIGNED;
+  st = check_device();
+  if (st != NB_OK) return st;
+  nb::AttnArgs a = make_args(q, k, v, o, nullptr, lse, lengths, nullptr, nullptr, nullptr,
+                             nullptr, batch, heads, n, d, R, causal);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e =
+      dtype == NB_F32 ? nb::launch_attn_fwd_f32(a, s) : nb::launch_attn_fwd_bf16_tc(a, s);
+  return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
+}
+
+nb_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                   const float* lse, const int32_t* lengths, void* dq, void* dk, void* dv,
+                   void* workspace, size_t workspace_bytes, int batch, int heads, int n, int d,
+                   int R, int dtype, void* stream, bool causal) {
+  nb_status st = check_shape(batch, heads, n, d, R, dtype);
+  if (st != NB_OK) return st;
+  if (static_cast<int64_t>(batch) * heads * n == 0) return NB_OK;
+  if (dtype != NB_BF16) return NB_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return NB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (lengths && (reinterpret_cast<uintptr_t>(lengths) & 3u)))
+    return NB_ERR_MISALIGNED;
+  const int64_t rows = static_cast<int64_t>(batch) * heads * n;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < nb::bwd_workspace_bytes(rows, d))
+    return NB_ERR_WORKSPACE;
+  st = check_device();
+  if (st != NB_OK) return st;
+  nb::AttnArgs a = make_args(q, k, v, o, dout, lse, lengths, dq, dk, dv, workspace, batch, heads,
+                             n, d, R, causal);
+  cudaError_t e = nb::launch_attn_bwd_bf16(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
 }
 
 }  // namespace
@@ -115,21 +162,13 @@ nb_status nb_kernel_error(int* code, int clear) {
 nb_status nb_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                       const int32_t* lengths, int batch, int heads, int n, int d, int R,
                       int dtype, void* stream) {
-  nb_status st = check_shape(batch, heads, n, d, R, dtype);
-  if (st != NB_OK) return st;
-  if (static_cast<int64_t>(batch) * heads * n == 0) return NB_OK;
-  if (!q || !k || !v || !o) return NB_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (lse && !aligned16(lse)) || (lengths && (reinterpret_cast<uintptr_t>(lengths) & 3u)))
-    return NB_ERR_MISALIGNED;
-  st = check_device();
-  if (st != NB_OK) return st;
-  nb::AttnArgs a = make_args(q, k, v, o, nullptr, lse, lengths, nullptr, nullptr, nullptr,
-                             nullptr, batch, heads, n, d, R);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e =
-      dtype == NB_F32 ? nb::launch_attn_fwd_f32(a, s) : nb::launch_attn_fwd_bf16_tc(a, s);
-  return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
+  return attn_fwd(q, k, v, o, lse, lengths, batch, heads, n, d, R, dtype, stream, false);
+}
+
+nb_status nb_attn_fwd_causal(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const int32_t* lengths, int batch, int heads, int n, int d, int R,
+                             int dtype, void* stream) {
+  return attn_fwd(q, k, v, o, lse, lengths, batch, heads, n, d, R, dtype, stream, true);
 }
 
 size_t nb_attn_bwd_workspace_size(int batch, int heads, int n, int d, int dtype) {
@@ -143,25 +182,16 @@ nb_status nb_attn_bwd(const void* q, const void* k, const void* v, const void* o
                       const void* dout, const float* lse, const int32_t* lengths, void* dq,
                       void* dk, void* dv, void* workspace, size_t workspace_bytes, int batch,
                       int heads, int n, int d, int R, int dtype, void* stream) {
-  nb_status st = check_shape(batch, heads, n, d, R, dtype);
-  if (st != NB_OK) return st;
-  if (static_cast<int64_t>(batch) * heads * n == 0) return NB_OK;
-  if (dtype != NB_BF16) return NB_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return NB_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
-      (lengths && (reinterpret_cast<uintptr_t>(lengths) & 3u)))
-    return NB_ERR_MISALIGNED;
-  const int64_t rows = static_cast<int64_t>(batch) * heads * n;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      workspace_bytes < nb::bwd_workspace_bytes(rows, d))
-    return NB_ERR_WORKSPACE;
-  st = check_device();
-  if (st != NB_OK) return st;
-  nb::AttnArgs a = make_args(q, k, v, o, dout, lse, lengths, dq, dk, dv, workspace, batch, heads,
-                             n, d, R);
-  cudaError_t e = nb::launch_attn_bwd_bf16(a, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
+  return attn_bwd(q, k, v, o, dout, lse, lengths, dq, dk, dv, workspace, workspace_bytes, batch,
+                  heads, n, d, R, dtype, stream, false);
+}
+
+nb_status nb_attn_bwd_causal(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, const int32_t* lengths, void* dq,
+                             void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                             int batch, int heads, int n, int d, int R, int dtype, void* stream) {
+  return attn_bwd(q, k, v, o, dout, lse, lengths, dq, dk, dv, workspace, workspace_bytes, batch,
+                  heads, n, d, R, dtype, stream, true);
 }
 
 nb_status nb_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,

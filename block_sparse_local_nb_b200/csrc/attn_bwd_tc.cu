@@ -115,7 +115,7 @@ __device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int ti
   x.nch = 0;
   if (x.tile * kRows < x.L) {
     const int kb_last = min(x.tile * 4 + 3, nb - 1);
-    x.I0 = max(0, x.tile * 4 - a.R);
+    x.I0 = a.causal ? x.tile * 4 : max(0, x.tile * 4 - a.R);  // causal: queries at or after the keys
     const int I1 = min(min(kb_last + a.R, nb - 1), (x.L - 1) / kBlock);
     x.nch = (I1 - x.I0 + 4) / 4;
   }
@@ -406,7 +406,10 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
         const float(&s)[32] = sa[jj];
         const float(&dp)[32] = dpa[jj];
         const int qb = x.I0 + 4 * c + j;
-        const bool vis = row_valid && qb < nb && abs(qb - kb) <= a.R;
+        const bool vis = row_valid && qb < nb &&
+                         (a.causal ? (qb >= kb && qb - kb <= a.R) : abs(qb - kb) <= a.R);
+        // causal, diagonal block: queries before this key (index < k mod 32) see it not
+        const int cut = a.causal && qb == kb ? (k & (kBlock - 1)) : 0;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           if (vis) {
@@ -421,8 +424,10 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
             const float2 sl = make_float2(sl2, sl2);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {  // pairs of queries, packed fp32x2 arithmetic
-              const float2 x = __ffma2_rn(make_float2(s[8 * cc + 2 * e], s[8 * cc + 2 * e + 1]),
-                                          sl, nv[e]);  // -inf for padding queries -> P = 0
+              float2 x = __ffma2_rn(make_float2(s[8 * cc + 2 * e], s[8 * cc + 2 * e + 1]),
+                                    sl, nv[e]);  // -inf for padding queries -> P = 0
+              if (8 * cc + 2 * e < cut) x.x = -INFINITY;
+              if (8 * cc + 2 * e + 1 < cut) x.y = -INFINITY;
               const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
               const float2 de = __fmul2_rn(
                   pe, __fadd2_rn(make_float2(dp[8 * cc + 2 * e], dp[8 * cc + 2 * e + 1]), nd[e]));

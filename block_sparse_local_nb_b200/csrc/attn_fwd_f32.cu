@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(AttnArgs a) {
   float m = -INFINITY, l = 0.f;
 
   const int jlast = (L - 1) / kBlock;  // last key block holding a valid key
-  const int j0 = max(0, qb - a.R), j1 = min(min(nb - 1, qb + a.R), jlast);
+  const int j0 = max(0, qb - a.R), j1 = min(min(nb - 1, qb + (a.causal ? 0 : a.R)), jlast);
   for (int j = j0; j <= j1; ++j) {
     const float4* ksrc = reinterpret_cast<const float4*>(kp + (int64_t)j * kBlock * D);
     const float4* vsrc = reinterpret_cast<const float4*>(vp + (int64_t)j * kBlock * D);
@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(AttnArgs a) {
       for (int i = 0; i < DPT; ++i) part = fmaf(qv[i], Ks[kk][sub + 4 * i], part);
       part += __shfl_xor_sync(0xffffffffu, part, 1);
       part += __shfl_xor_sync(0xffffffffu, part, 2);
-      s[kk] = (j * kBlock + kk < L) ? part : -INFINITY;
+      const int key = j * kBlock + kk;  // keys past the length (or, causal, after the query) masked
+      s[kk] = (key < L && (!a.causal || key <= qrow)) ? part : -INFINITY;
       mblk = fmaxf(mblk, s[kk]);
     }
     const float mnew = fmaxf(m, mblk);

@@ -115,7 +115,7 @@ __device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int ti
   if (x.tile * kRows < x.L) {
     const int qb_last = min(x.tile * 4 + 3, nb - 1);
     x.J0 = max(0, x.tile * 4 - a.R);
-    const int J1 = min(min(qb_last + a.R, nb - 1), (x.L - 1) / kBlock);
+    const int J1 = min(min(qb_last + (a.causal ? 0 : a.R), nb - 1), (x.L - 1) / kBlock);
     x.nch = (J1 - x.J0 + 4) / 4;
   }
   return x;
@@ -379,9 +379,11 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int kb = x.J0 + 4 * c + 2 * hf + j;
-        vis[j] = row_valid && kb < nb && abs(kb - qb) <= a.R && kb * kBlock < x.L;
+        vis[j] = row_valid && kb < nb && kb * kBlock < x.L &&
+                 (a.causal ? (kb <= qb && qb - kb <= a.R) : abs(kb - qb) <= a.R);
         if (vis[j]) {
-          const int lim = x.L - kb * kBlock;  // keys at or past the length are masked
+          // keys at or past the length are masked, and (causal) keys after the query
+          const int lim = min(x.L - kb * kBlock, a.causal && kb == qb ? q - kb * kBlock + 1 : kBlock);
           if (lim < 32) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) s[j][i] = i < lim ? s[j][i] : -INFINITY;

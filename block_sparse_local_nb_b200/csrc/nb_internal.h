@@ -25,6 +25,7 @@ struct AttnArgs {
   int* err;           // device word receiving the first wait-timeout code (may be null)
   int batch, heads, n, d, R;
   float scale;        // 1/sqrt(d)
+  bool causal;        // causal band: key blocks i - R..i of query block i, keys k <= q
 };
 
 size_t bwd_workspace_bytes(int64_t rows, int d);

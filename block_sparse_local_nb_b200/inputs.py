@@ -41,6 +41,7 @@ class AttnWorkload:
     varlen: tuple | None = None  # (lo, hi) inclusive range of sequence lengths
     backward: bool = True
     desc: str = field(default="", compare=False)
+    causal: bool = False  # the causal band (key blocks i - R..i, keys k <= q)
 
 
 WORKLOADS = {
@@ -48,6 +49,10 @@ WORKLOADS = {
                               desc="fwd fp32 1x1x256x64 R=1 full"),
     "bf16_varlen": AttnWorkload("bf16_varlen", "bf16", 4, 12, 4096, 64, 2, 2, varlen=(1024, 4096),
                                 desc="fwd+bwd bf16 4x12x4096x64 R=2 L~U[1024,4096]"),
+    "bf16_varlen_causal": AttnWorkload("bf16_varlen_causal", "bf16", 4, 12, 4096, 64, 2, 2,
+                                       varlen=(1024, 4096), causal=True,
+                                       desc="fwd+bwd bf16 4x12x4096x64 R=2 causal band "
+                                            "L~U[1024,4096]"),
     "bf16_n131k": AttnWorkload("bf16_n131k", "bf16", 1, 16, 131072, 128, 4, 3, scale=0.5,
                                desc="fwd+bwd bf16 1x16x131072x128 R=4 full"),
     "bf16_n1m": AttnWorkload("bf16_n1m", "bf16", 1, 8, 1048576, 64, 8, 4,

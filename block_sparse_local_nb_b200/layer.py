@@ -72,10 +72,11 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 class BlockSparseLocalAttention(torch.autograd.Function):
     """O = softmax(Q K^T / sqrt(d) restricted to the band |i - j| <= R of
-    32-token blocks and to keys < lengths[b]) V, with its backward."""
+    32-token blocks and to keys < lengths[b]) V, with its backward.  With
+    ``causal`` the band is i - R <= j <= i and keys k <= q."""
 
     @staticmethod
-    def forward(ctx, q, k, v, lengths, R: int):
+    def forward(ctx, q, k, v, lengths, R: int, causal: bool = False):
         if not (q.shape == k.shape == v.shape and q.dim() == 4):
             raise ValueError("q, k, v must share one [batch, heads, n, d] shape")
         if not (q.dtype == k.dtype == v.dtype):
@@ -86,10 +87,12 @@ class BlockSparseLocalAttention(torch.autograd.Function):
             lengths = lengths.to(device=q.device, dtype=torch.int32).contiguous()
         o = torch.empty_like(q)
         lse = torch.empty((batch, heads, n), dtype=torch.float32, device=q.device)
-        nb.nb_attn_fwd(q, k, v, o, lse, lengths, batch, heads, n, d, R, _dtype_code(q),
-                       torch.cuda.current_stream(q.device))
+        fwd = nb.nb_attn_fwd_causal if causal else nb.nb_attn_fwd
+        fwd(q, k, v, o, lse, lengths, batch, heads, n, d, R, _dtype_code(q),
+            torch.cuda.current_stream(q.device))
         ctx.save_for_backward(q, k, v, o, lse, lengths)
         ctx.R = R
+        ctx.causal = causal
         return o
 
     @staticmethod
@@ -101,11 +104,12 @@ class BlockSparseLocalAttention(torch.autograd.Function):
         ws_bytes = nb.attn_bwd_workspace_size(batch, heads, n, d, code)
         ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        nb.nb_attn_bwd(q, k, v, o, do, lse, lengths, dq, dk, dv, ws, ws_bytes, batch, heads, n, d,
-                       ctx.R, code, torch.cuda.current_stream(q.device))
-        return dq, dk, dv, None, None
+        bwd = nb.nb_attn_bwd_causal if ctx.causal else nb.nb_attn_bwd
+        bwd(q, k, v, o, do, lse, lengths, dq, dk, dv, ws, ws_bytes, batch, heads, n, d, ctx.R, code,
+            torch.cuda.current_stream(q.device))
+        return dq, dk, dv, None, None, None
 
 
-def block_sparse_local_attention(q, k, v, lengths=None, R: int = 1):
+def block_sparse_local_attention(q, k, v, lengths=None, R: int = 1, causal: bool = False):
     """Differentiable banded block-sparse local attention (see the class)."""
-    return BlockSparseLocalAttention.apply(q, k, v, lengths, R)
+    return BlockSparseLocalAttention.apply(q, k, v, lengths, R, causal)

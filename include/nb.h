@@ -134,6 +134,23 @@ NB_API nb_status nb_attn_bwd(const void* q, const void* k, const void* v, const 
                       int heads, int n, int d, int R, int dtype, void* stream);
 
 /*
+ * nb_attn_fwd_causal / nb_attn_bwd_causal - the causal band.  The NucleoByte
+ * page's band is symmetric; this is its causal restriction (the plainest
+ * reading of a causal band, a variant the page does not print): query q in
+ * block i attends key k in block j only when i - R <= j <= i and k <= q (and
+ * k < L_b).  Same arguments, layouts, workspace and errors as nb_attn_fwd /
+ * nb_attn_bwd; the fp32 forward is supported, the backward is bf16 only.
+ */
+NB_API nb_status nb_attn_fwd_causal(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, const int32_t* lengths, int batch, int heads,
+                                    int n, int d, int R, int dtype, void* stream);
+NB_API nb_status nb_attn_bwd_causal(const void* q, const void* k, const void* v, const void* o,
+                                    const void* dout, const float* lse, const int32_t* lengths,
+                                    void* dq, void* dk, void* dv, void* workspace,
+                                    size_t workspace_bytes, int batch, int heads, int n, int d,
+                                    int R, int dtype, void* stream);
+
+/*
  * nb_attn_bwd_noalloc - nb_attn_bwd for callers that cannot allocate device
  * memory.  The NucleoByte page has no counterpart: it exists for callers that
  * cannot hand the library a workspace, such as a host program whose device

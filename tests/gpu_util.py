@@ -17,25 +17,27 @@ def dtype_code(t: torch.dtype) -> int:
     return nb.NB_F32 if t == torch.float32 else nb.NB_BF16
 
 
-def run_fwd(q, k, v, lengths, R, with_lse=True):
-    """Forward through nb_attn_fwd; returns (o, lse) device tensors."""
+def run_fwd(q, k, v, lengths, R, with_lse=True, causal=False):
+    """Forward through nb_attn_fwd (or nb_attn_fwd_causal); returns (o, lse) device tensors."""
     batch, heads, n, d = q.shape
     o = torch.empty_like(q)
     lse = torch.empty((batch, heads, n), device=q.device, dtype=torch.float32) if with_lse else None
     lens = None if lengths is None else lengths.to(device=q.device, dtype=torch.int32)
-    nb.nb_attn_fwd(q, k, v, o, lse, lens, batch, heads, n, d, R, dtype_code(q.dtype))
+    fwd = nb.nb_attn_fwd_causal if causal else nb.nb_attn_fwd
+    fwd(q, k, v, o, lse, lens, batch, heads, n, d, R, dtype_code(q.dtype))
     return o, lse
 
 
-def run_bwd(q, k, v, o, do, lse, lengths, R, workspace=None):
+def run_bwd(q, k, v, o, do, lse, lengths, R, workspace=None, causal=False):
     batch, heads, n, d = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws_bytes = nb.attn_bwd_workspace_size(batch, heads, n, d, dtype_code(q.dtype))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     lens = None if lengths is None else lengths.to(device=q.device, dtype=torch.int32)
-    nb.nb_attn_bwd(q, k, v, o, do, lse, lens, dq, dk, dv, workspace, ws_bytes, batch, heads, n,
-                   d, R, dtype_code(q.dtype))
+    bwd = nb.nb_attn_bwd_causal if causal else nb.nb_attn_bwd
+    bwd(q, k, v, o, do, lse, lens, dq, dk, dv, workspace, ws_bytes, batch, heads, n, d, R,
+        dtype_code(q.dtype))
     return dq, dk, dv
 
 

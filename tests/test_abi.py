@@ -158,3 +158,25 @@ def test_tokenize_batch_rejects_invalid_arguments(lib, kw, status):
     args.update(kw)
     assert lib.nb_tokenize_batch(args["seqs"], args["offsets"], args["batch"], args["k"], args["ids"],
                                  args["lengths"], args["n_pad"], None) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n=48), NB_ERR_INVALID_ARG), (dict(R=-1), NB_ERR_INVALID_ARG), (dict(d=96), NB_ERR_UNSUPPORTED),
+    (dict(k=24), NB_ERR_MISALIGNED), (dict(batch=0), NB_OK),
+])
+def test_causal_entry_points_validate_like_the_band(lib, kw, status):
+    args = dict(q=16, k=16, v=16, o=16, lse=None, lengths=None, batch=1, heads=1, n=64, d=64, R=1,
+                dtype=BF16)
+    args.update(kw)
+    a = args
+    assert lib.nb_attn_fwd_causal(a["q"], a["k"], a["v"], a["o"], a["lse"], a["lengths"], a["batch"],
+                                  a["heads"], a["n"], a["d"], a["R"], a["dtype"], None) == status
+    st = lib.nb_attn_bwd_causal(a["q"], a["k"], a["v"], a["o"], 16, 16, None, 16, 16, 16, 256,
+                                1 << 30, a["batch"], a["heads"], a["n"], a["d"], a["R"], a["dtype"],
+                                None)
+    assert st == status
+
+
+def test_causal_backward_rejects_fp32(lib):
+    assert lib.nb_attn_bwd_causal(16, 16, 16, 16, 16, 16, None, 16, 16, 16, 256, 1 << 30, 1, 1, 64,
+                                  64, 1, F32, None) == NB_ERR_UNSUPPORTED

@@ -9,18 +9,19 @@ from block_sparse_local_nb_b200.inputs import AttnWorkload
 from oracle.attention import block_band_mask
 
 
+@pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("n,R,lengths,heads,d,dtype", [
     (256, 1, [256], 1, 64, "f32"),
     (512, 2, [512, 333, 1, 0], 3, 64, "bf16"),
     (320, 0, [300, 32], 2, 128, "bf16"),
     (256, 9, [256, 200], 1, 64, "bf16"),  # band wider than the sequence
 ])
-def test_algorithmic_units_match_brute_force(n, R, lengths, heads, d, dtype):
-    w = AttnWorkload("t", dtype, len(lengths), heads, n, d, R, 0)
+def test_algorithmic_units_match_brute_force(n, R, lengths, heads, d, dtype, causal):
+    w = AttnWorkload("t", dtype, len(lengths), heads, n, d, R, 0, causal=causal)
     alg = bench.algorithmic(w, lengths)
     pairs = 0
     for L in lengths:
-        m = block_band_mask(n, R, L)[:L]  # valid query rows, visible keys
+        m = block_band_mask(n, R, L, causal=causal)[:L]  # valid query rows, visible keys
         pairs += int(m.sum())
     e = 4 if dtype == "f32" else 2
     th = sum(lengths) * heads

@@ -81,3 +81,17 @@ def test_collate_feeds_attention_end_to_end():
     assert torch.isfinite(emb.weight.grad.float()).all()
     for row, L in enumerate(lengths.cpu().tolist()):
         assert (o[row, :, L:] == 0).all()
+
+
+def test_autograd_causal_matches_direct_calls():
+    q, k, v, do = (t.cuda() for t in random_attn_inputs(2, 2, 384, 64, "bf16", seed=41))
+    L = torch.tensor([384, 250], dtype=torch.int32)
+    qa, ka, va = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o = block_sparse_local_attention(qa, ka, va, L.cuda(), 2, causal=True)
+    o.backward(do)
+    o_ref, lse = run_fwd(q, k, v, L, 2, causal=True)
+    dq, dk, dv = run_bwd(q, k, v, o_ref, do, lse, L, 2, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref)
+    assert torch.equal(ka.grad, dk) and torch.equal(va.grad, dv)
+    assert rel_fro(f64(qa.grad), f64(dq)) < 1e-3

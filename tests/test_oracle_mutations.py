@@ -170,6 +170,7 @@ CAUSAL_MUTATIONS = [
 ]
 
 
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")  # the mutants' own arithmetic
 @pytest.mark.parametrize("name,old,new", CAUSAL_MUTATIONS, ids=[m[0] for m in CAUSAL_MUTATIONS])
 def test_causal_mutation_is_caught(name, old, new):
     assert old in SRC_ATT, name

@@ -311,7 +311,7 @@ __device__ int out_storer(const Params& p, const Sched& sch, uint32_t base, cons
 }
 
 // Gradient warps: thread = key row r; half hf owns query columns [64 hf, 64 hf + 64).
-template <int D>
+template <int D, bool kCausal>
 __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
                           uint32_t tmem, int wq, int hf, int lane) {
   using C = Cfg<D>;
@@ -407,9 +407,9 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
         const float(&dp)[32] = dpa[jj];
         const int qb = x.I0 + 4 * c + j;
         const bool vis = row_valid && qb < nb &&
-                         (a.causal ? (qb >= kb && qb - kb <= a.R) : abs(qb - kb) <= a.R);
+                         (kCausal ? (qb >= kb && qb - kb <= a.R) : abs(qb - kb) <= a.R);
         // causal, diagonal block: queries before this key (index < k mod 32) see it not
-        const int cut = a.causal && qb == kb ? (k & (kBlock - 1)) : 0;
+        const int cut = kCausal && qb == kb ? (k & (kBlock - 1)) : 0;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           if (vis) {
@@ -558,7 +558,7 @@ __device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint8_
   return 0;
 }
 
-template <int D>
+template <int D, bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                        const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
@@ -642,7 +642,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 12) {
     regs_inc<C::kRegsGrad>();
-    const int err = grad_warps<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
+    const int err =
+        grad_warps<D, kCausal>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
     if (err) record_error(p.a.err, err);
     pdl_trigger();  // this CTA's work is issued: the next kernel may start launching
     __syncthreads();
@@ -675,11 +676,12 @@ cudaError_t launch(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
   const int64_t items = heads_total * p.ntiles;
   if (items > (1ll << 30)) return cudaErrorInvalidValue;
   p.items = static_cast<int>(items);
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  auto kernel = a.causal ? attn_bwd_tc_kernel<D, true> : attn_bwd_tc_kernel<D, false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  return launch_pdl(attn_bwd_tc_kernel<D>, dim3(grid), dim3(kThreads), C::kSmem, stream, tk, tv, tq,
+  return launch_pdl(kernel, dim3(grid), dim3(kThreads), C::kSmem, stream, tk, tv, tq,
                     tdo, tdq, tdk, tdv, p);
 }
 

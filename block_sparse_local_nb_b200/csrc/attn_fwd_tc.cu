@@ -251,7 +251,7 @@ __device__ int pv_issuer(const Params& p, const Sched& sch, uint32_t base, uint3
   return 0;
 }
 
-template <int D>
+template <int D, bool kCausal>
 __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
                                 uint32_t tmem, int wq, int hf, int lane, const CUtensorMap* to) {
   using C = Cfg<D>;
@@ -380,10 +380,10 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
       for (int j = 0; j < 2; ++j) {
         const int kb = x.J0 + 4 * c + 2 * hf + j;
         vis[j] = row_valid && kb < nb && kb * kBlock < x.L &&
-                 (a.causal ? (kb <= qb && qb - kb <= a.R) : abs(kb - qb) <= a.R);
+                 (kCausal ? (kb <= qb && qb - kb <= a.R) : abs(kb - qb) <= a.R);
         if (vis[j]) {
           // keys at or past the length are masked, and (causal) keys after the query
-          const int lim = min(x.L - kb * kBlock, a.causal && kb == qb ? q - kb * kBlock + 1 : kBlock);
+          const int lim = min(x.L - kb * kBlock, kCausal && kb == qb ? q - kb * kBlock + 1 : kBlock);
           if (lim < 32) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) s[j][i] = i < lim ? s[j][i] : -INFINITY;
@@ -472,7 +472,7 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
   return 0;
 }
 
-template <int D>
+template <int D, bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
@@ -538,7 +538,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 10) {
     if (lane == 0) err = pv_issuer<D>(p, sch, base, tmem);
   } else {
-    err = softmax_epilogue<D>(p, sch, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane, &to);
+    err = softmax_epilogue<D, kCausal>(p, sch, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane,
+                                       &to);
   }
   if (err) record_error(p.a.err, err);
 
@@ -572,11 +573,12 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
   const int64_t items = heads_total * p.ntiles;
   if (items > (1ll << 30)) return cudaErrorInvalidValue;
   p.items = static_cast<int>(items);
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  auto kernel = a.causal ? attn_fwd_tc_kernel<D, true> : attn_fwd_tc_kernel<D, false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
-  return launch_pdl(attn_fwd_tc_kernel<D>, dim3(grid), dim3(kThreads), C::kSmem, stream, tq, tk, tv,
+  return launch_pdl(kernel, dim3(grid), dim3(kThreads), C::kSmem, stream, tq, tk, tv,
                     to, p);
 }
 

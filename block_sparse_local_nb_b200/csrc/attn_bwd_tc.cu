@@ -5,6 +5,8 @@
 // shared key/value blocks accumulated with atomic adds.)
 //
 // Work item = one key tile of 128 keys (four key blocks) of one (batch, head).
+// (The causal band, the kCausal instantiation, takes query blocks 4t ..
+// 4t + 3 + R and zeroes P for queries before their key in the diagonal block.)
 // The band is symmetric, so its dK and dV need only the query blocks
 // [4t - R, 4t + 3 + R], taken in chunks of 128 queries.  Per chunk, with keys
 // on the TMEM lanes (M = 128):

@@ -7,7 +7,9 @@
 // give, so this path uses FFMA.  One CTA of 128 threads owns one query block
 // (32 rows): four threads per row, each holding d/4 interleaved dimensions of
 // the query and of the output accumulator.  The key and value blocks of the
-// band are staged through shared memory one block at a time.
+// band are staged through shared memory one block at a time.  With the causal
+// band (a.causal) the window is blocks qb - R .. qb and keys after the query
+// are masked.
 #include <math.h>
 
 #include "nb_internal.h"

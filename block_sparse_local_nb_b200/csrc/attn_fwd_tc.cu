@@ -5,7 +5,9 @@
 //
 // Work item = one query tile of 128 rows (four query blocks) of one (batch,
 // head).  The union of the four bands is the key-block window
-// [4t - R, 4t + 3 + R] (clipped to the sequence and its length), processed in
+// [4t - R, 4t + 3 + R] ([4t - R, 4t + 3] for the causal band, the kCausal
+// instantiation, which also masks keys after their query in the diagonal
+// block) (clipped to the sequence and its length), processed in
 // chunks of 128 keys (four key blocks).  A persistent grid of one CTA per SM
 // walks the items; consecutive CTAs take neighbouring tiles at the same time,
 // so the key/value blocks their windows share are served from L2.

@@ -177,13 +177,13 @@ def _check_window(w, tensors, outs, bh, blk_lo, blk_hi, lengths, check_bwd=True)
     Lsub = min(max(Lb - s * BLOCK, 0), (e - s) * BLOCK)
     sl = slice(s * BLOCK, e * BLOCK)
     sub = [t[b, h, sl].double().cpu().numpy()[None, None] for t in (q, k, v, do)]
-    o_ref, lse_ref = attn_fwd_banded(*sub[:3], w.R, [Lsub])
+    o_ref, lse_ref = attn_fwd_banded(*sub[:3], w.R, [Lsub], causal=w.causal)
     r0, r1 = (blk_lo - s) * BLOCK, (blk_hi - s) * BLOCK
     g0, g1 = blk_lo * BLOCK, blk_hi * BLOCK
     assert max_abs(f64(o[b, h, g0:g1]), o_ref[0, 0, r0:r1]) <= O_ATOL_BF16
     assert max_abs(f64(lse[b, h, g0:g1]), lse_ref[0, 0, r0:r1]) <= LSE_ATOL_BF16
     if check_bwd:
-        grads_ref = attn_bwd_banded(*sub, w.R, [Lsub])
+        grads_ref = attn_bwd_banded(*sub, w.R, [Lsub], causal=w.causal)
         for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), grads_ref):
             err = rel_fro(f64(g[b, h, g0:g1]), r[0, 0, r0:r1])
             assert err <= GRAD_RFRO_BF16, (name, err)
@@ -191,16 +191,19 @@ def _check_window(w, tensors, outs, bh, blk_lo, blk_hi, lengths, check_bwd=True)
 
 def _run_workload(w):
     q, k, v, do, lengths = make_attn_inputs(w, device="cuda")
-    o, lse = run_fwd(q, k, v, lengths, w.R)
-    grads = run_bwd(q, k, v, o, do, lse, lengths, w.R) if w.backward else (None,) * 3
+    o, lse = run_fwd(q, k, v, lengths, w.R, causal=w.causal)
+    grads = run_bwd(q, k, v, o, do, lse, lengths, w.R, causal=w.causal) if w.backward else (None,) * 3
     torch.cuda.synchronize()
     return (q, k, v, do), (o, lse, *grads), lengths
 
 
-def test_bf16_varlen_workload():
-    """bf16, 4 x 12 x 4096 x 64, R = 2, lengths ~ U[1024, 4096]: three whole heads
-    and sampled windows of the rest, including each sequence's length boundary."""
-    w = WORKLOADS["bf16_varlen"]
+@pytest.mark.parametrize("name", ["bf16_varlen", "bf16_varlen_causal"])
+def test_bf16_varlen_workload(name):
+    """bf16, 4 x 12 x 4096 x 64, R = 2, lengths ~ U[1024, 4096] (symmetric and
+    causal band): three whole heads and sampled windows of the rest, including
+    each sequence's length boundary.  The windows carry 2R blocks of context on
+    each side, which covers every dependency of the checked blocks in both bands."""
+    w = WORKLOADS[name]
     tensors, outs, lengths = _run_workload(w)
     nb = w.n // BLOCK
     for bh in [(0, 0), (1, 5), (3, 11)]:

@@ -4,15 +4,20 @@ block-sparse local attention forward + backward, through the C ABI.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 One step = one pass of every step of the path over one batch: nb_tokenize_kmer
-on the batch's DNA (batch x (n + 5) bases), nb_attn_fwd and nb_attn_bwd.  Inputs
-are seeded synthetic tensors resident in HBM; several input sets rotate so that
-each step reads inputs that are not L2-resident.  Time is taken with CUDA
-events on the launching stream, bracketed by a barrier and a device
+on the batch's DNA (batch x (n + 5) bases), nb_attn_fwd and nb_attn_bwd.  The
+headline workload is the largest single-GPU configuration, ``bf16_n1m``
+(1 x 8 x 1048576 x 64, R = 8: the forward, then forward + backward).  Inputs
+are seeded synthetic tensors resident in HBM; several input sets rotate so
+that each step reads inputs that are not L2-resident.  Time is taken with
+CUDA events on the launching stream, bracketed by a barrier and a device
 synchronize, and the max over ranks is reported.  For N > 1 every rank
 processes its own batch (weak scaling, no collective on the data path).
 
-Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle (fp64
-NumPy) on a bounded sample of the same workload instead.
+Rank 0 prints one JSON line.  At N = 1 the line also carries ``sub_results``:
+the other configurations (fp32 1 x 1 x 256, the ragged-length bf16 batch,
+the 131072-token d = 128 sequence and the 2**28-base tokenizer), each timed
+the same way with its own roofline.  ``--impl reference`` times the CPU
+oracle (fp64 NumPy) on a bounded sample of the same workload instead.
 """
 
 from __future__ import annotations
@@ -31,8 +36,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "block-sparse local attn fwd+bwd tokens/s and % of roofline (HBM or tensor)"
+HEADLINE = "bf16_n1m"
+SUB_WORKLOADS = ("fp32_n256", "bf16_varlen", "bf16_n131k", "dna_2p28")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
+SUSTAINED_AFTER_S = 2.0  # a timed region at least this long is compared with the sustained peak
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic.json")
 
 
 # ----------------------------------------------------------------- helpers
@@ -66,20 +75,20 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch recorded from an ncu capture in profiles/, valid
-    only while the kernel sources still hash to the value recorded with it."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    """DRAM bytes (read + write) per launch of `kernel` on `workload`, from the
+    JSON record of ncu captures, valid only while the kernel sources still hash
+    to the value recorded with it (else None)."""
     try:
-        lines = open(path).read().splitlines()
-    except OSError:
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
     src = kernel_source_hash()
-    for line in lines:
-        parts = [p.strip() for p in line.strip().strip("|").split("|")]
-        if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[3] == src:
+    for r in rec.get("records", []):
+        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("source_hash") == src:
             try:
-                return float(parts[2])
-            except ValueError:
+                return float(r["bytes_per_launch"])
+            except (KeyError, TypeError, ValueError):
                 return None
     return None
 
@@ -94,6 +103,7 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.proc = None
         self.device_index = device_index
+        self.lines = []
 
     def __enter__(self):
         try:
@@ -178,150 +188,388 @@ def algorithmic(w, lengths):
     }
 
 
+def tokenizer_bytes(bases: int, k: int = 6) -> int:
+    """Algorithmic bytes of nb_tokenize_kmer: 1 byte read per base, a uint16 ID
+    written per window and the packed stream (one byte per four bases)."""
+    return bases + 2 * max(bases - k + 1, 0) + (bases + 3) // 4
+
+
 def dna_for_batch(w, seed):
     from block_sparse_local_nb_b200.inputs import make_dna
 
     return make_dna(w.batch * (w.n + 5), seed=seed)
 
 
-def run_reference_arm(args, w):
-    """Time the CPU oracle on a bounded sample of the workload (rank 0 only)."""
-    import numpy as np
-    from threadpoolctl import threadpool_info
+def fp32_peak_tflops(sm_mhz):
+    """CUDA-core fp32 FMA peak: SMs x 128 lanes x 2 flops x clock."""
+    import torch
 
-    from block_sparse_local_nb_b200.inputs import make_attn_inputs
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return sms * 128 * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12
+
+
+def roofline(nbytes, flops, ms, peaks, timed_s, dtype, sm_max_mhz=None):
+    """Fraction of the roofline of one call: the slower of its algorithmic
+    bytes at HBM bandwidth and its algorithmic flops at the tensor (bf16) or
+    fp32 FMA peak.  The bf16 peak is the burst figure for a timed region
+    shorter than SUSTAINED_AFTER_S seconds, else the sustained figure."""
+    hbm = float(peaks["hbm_gbs"])
+    if dtype == "bf16":
+        sustained = timed_s >= SUSTAINED_AFTER_S and "bf16_tflops_sustained" in peaks
+        comp = float(peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"])
+        comp_bound, comp_kind = "tensor", "sustained" if sustained else "burst"
+    else:
+        comp = fp32_peak_tflops(sm_max_mhz)
+        comp_bound, comp_kind = "alu", "fp32 FMA: SMs x 128 x 2 x max SM clock"
+    t_hbm = nbytes / (hbm * 1e9)
+    t_comp = flops / (comp * 1e12)
+    if t_hbm >= t_comp:
+        achieved = nbytes / (ms / 1e3) / 1e9
+        r = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s"}
+    else:
+        achieved = flops / (ms / 1e3) / 1e12
+        r = {"bound": comp_bound, "achieved": achieved, "peak": comp, "unit": "TFLOP/s",
+             "peak_kind": comp_kind}
+    r["frac"] = r["achieved"] / r["peak"]
+    r["roofline_ms"] = max(t_hbm, t_comp) * 1e3
+    return r
+
+
+# ------------------------------------------------------- oracle samples
+
+def oracle_window(w, lengths, step):
+    """(sequence, head, first block, end block) of the oracle sample of `step`:
+    a whole sequence when it has at most 256 blocks, else a window of 256
+    query blocks at a position that moves from step to step."""
+    nb_ = w.n // 32
+    b = step % w.batch
+    h = (step // w.batch) % w.heads
+    Lb = int(lengths[b])
+    blocks = (Lb + 31) // 32
+    if blocks <= 256:
+        return b, h, 0, blocks
+    lo = (step * 7919 * 32) % (blocks - 256 + 1)
+    return b, h, lo, min(nb_, lo + 256)
+
+
+def oracle_sample(w, fetch, lengths, dna, step):
+    """Run the fp64 oracle (forward, backward, tokenization) on one sample and
+    return the token-equivalents it covered (query rows of one head / heads).
+    A window is evaluated with two band radii of context on each side, where
+    the oracle's outputs for the window are exact.  ``fetch(b, h, r0, r1)``
+    returns rows [r0, r1) of Q, K, V, dO of one head as fp64 [1, 1, rows, d]."""
     from oracle import attn_bwd_banded, attn_fwd_banded, kmer_ids, pack_2bit
 
+    b, h, lo, hi = oracle_window(w, lengths, step)
+    nb_ = w.n // 32
+    s, e = max(0, lo - 2 * w.R), min(nb_, hi + 2 * w.R)
+    Lb = int(lengths[b])
+    Lsub = min(max(Lb - 32 * s, 0), 32 * (e - s))
+    sub = fetch(b, h, 32 * s, 32 * e)
+    attn_fwd_banded(*sub[:3], w.R, [Lsub], causal=w.causal)
+    if w.backward:
+        attn_bwd_banded(*sub, w.R, [Lsub], causal=w.causal)
+    rows = max(0, min(Lb, 32 * hi) - 32 * lo)
+    seg = dna[b * (w.n + 5) + 32 * lo: b * (w.n + 5) + 32 * lo + rows + 5]
+    kmer_ids(seg, 6)
+    pack_2bit(seg)
+    return rows / w.heads
+
+
+def window_fetcher(tensors):
+    """fetch(b, h, r0, r1) over [batch, heads, n, d] tensors (CPU or device)."""
+    def fetch(b, h, r0, r1):
+        return [t[b:b + 1, h:h + 1, r0:r1].to("cpu", copy=True).double().numpy() for t in tensors]
+    return fetch
+
+
+def _blas_threads():
+    from threadpoolctl import threadpool_info
+
+    return max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+
+
+def run_reference_arm(args, w):
+    """Time the CPU oracle on a bounded sample of the workload (rank 0 only)."""
+    from block_sparse_local_nb_b200.inputs import make_attn_inputs
+
     q, k, v, do, lengths = make_attn_inputs(w)
-    dna = dna_for_batch(w, seed=w.seed)
+    fetch = window_fetcher((q, k, v, do))
     lengths = lengths.numpy()
-    qn, kn, vn, don = (t.double().numpy() for t in (q, k, v, do))
-
-    def one(step):
-        # sample: one head of one sequence (rotating), plus that sequence's tokenization
-        b = step % w.batch
-        h = (step // w.batch) % w.heads
-        sl = (slice(b, b + 1), slice(h, h + 1))
-        Lb = [int(lengths[b])]
-        attn_fwd_banded(qn[sl], kn[sl], vn[sl], w.R, Lb, causal=w.causal)
-        attn_bwd_banded(qn[sl], kn[sl], vn[sl], don[sl], w.R, Lb, causal=w.causal)
-        seg = dna[b * (w.n + 5):(b + 1) * (w.n + 5)]
-        kmer_ids(seg, 6)
-        pack_2bit(seg)
-        return Lb[0] / w.heads  # token-equivalents (a token = all heads of one position)
-
+    dna = dna_for_batch(w, seed=w.seed)
     for s in range(args.warmup):
-        one(s)
+        oracle_sample(w, fetch, lengths, dna, s)
     t0 = time.perf_counter()
     tok = 0.0
     for s in range(args.steps):
-        tok += one(args.warmup + s)
+        tok += oracle_sample(w, fetch, lengths, dna, args.warmup + s)
     dt = time.perf_counter() - t0
     value = tok / dt
-    threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    cores = _blas_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "desc": w.desc, "batch": w.batch, "heads": w.heads,
-                   "n": w.n, "d": w.d, "R": w.R},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": "per step: one (sequence, head) of the batch through the fp64 "
-                                   "banded oracle forward+backward plus that sequence's k-mer "
-                                   "tokenization; counted as length/heads tokens"},
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "per step: one head of one sequence (whole when at most 256 "
+                                   "blocks, else a 256-block window of query blocks at a moving "
+                                   "position, evaluated with 2R blocks of context on each side) "
+                                   "through the fp64 banded oracle forward+backward plus the "
+                                   "k-mer tokenization of its bases; counted as rows/heads tokens"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(w):
-    """Oracle timed on the host cores on a bounded sample (~10 s of CPU work)."""
-    import numpy as np
-    from threadpoolctl import threadpool_info
-
-    from block_sparse_local_nb_b200.inputs import make_attn_inputs
-    from oracle import attn_bwd_banded, attn_fwd_banded, kmer_ids, pack_2bit
-
-    q, k, v, do, lengths = make_attn_inputs(w)
-    lengths = lengths.numpy()
-    dna = dna_for_batch(w, seed=w.seed)
-    qn, kn, vn, don = (t.double().numpy() for t in (q, k, v, do))
+def cpu_baseline(w, fetch, lengths, dna, budget_s=10.0):
+    """Oracle timed on the host cores on a bounded sample (about `budget_s` of
+    CPU work) of the benchmarked inputs."""
     t0 = time.perf_counter()
     tok = 0.0
-    heads_done = 0
-    pairs = w.batch * w.heads
-    budget = 10.0  # seconds; the pairs are cycled until the budget is spent
-    while time.perf_counter() - t0 < budget:
-        b, h = heads_done % w.batch, (heads_done // w.batch) % w.heads
-        sl = (slice(b, b + 1), slice(h, h + 1))
-        Lb = [int(lengths[b])]
-        attn_fwd_banded(qn[sl], kn[sl], vn[sl], w.R, Lb, causal=w.causal)
-        attn_bwd_banded(qn[sl], kn[sl], vn[sl], don[sl], w.R, Lb, causal=w.causal)
-        if h == 0:
-            seg = dna[b * (w.n + 5):(b + 1) * (w.n + 5)]
-            kmer_ids(seg, 6)
-            pack_2bit(seg)
-        tok += Lb[0] / w.heads
-        heads_done += 1
+    samples = 0
+    while time.perf_counter() - t0 < budget_s:
+        tok += oracle_sample(w, fetch, lengths, dna, samples)
+        samples += 1
     dt = time.perf_counter() - t0
-    threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
-    return {"value": tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{heads_done} (sequence, head) pairs ({heads_done / pairs:.2f} passes over "
-                      f"the workload's {pairs}) through the fp64 banded oracle fwd+bwd plus "
-                      f"per-sequence k-mer tokenization, {dt:.1f} s; host has "
-                      f"{os.cpu_count()} logical cores"}
+    return {"value": tok / dt, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{samples} samples in {dt:.1f} s, each one head of one sequence (whole when "
+                      f"at most 256 blocks, else a 256-block window of query blocks with 2R "
+                      f"blocks of context each side) through the fp64 banded oracle fwd+bwd plus "
+                      f"the k-mer tokenization of its bases, counted as rows/heads tokens; host "
+                      f"has {os.cpu_count()} logical cores"}
 
 
-def run_tokenizer_workload(args):
-    """The 2**28-byte k-mer tokenizer workload alone (one GPU): bases/s and the
-    fraction of the HBM roofline (1 byte read + 2.25 bytes written per base)."""
+def workload_config(w):
+    return {"workload": w.name, "desc": w.desc + " + k=6 tokenization of the batch's "
+            f"{w.batch}x({w.n}+5) bases", "batch": w.batch, "heads": w.heads, "n": w.n,
+            "d": w.d, "R": w.R}
+
+
+# ------------------------------------------------------------ GPU timing
+
+def time_attention(w, args, dev, rank, world, with_e2e, steps, warmup):
+    """Time `steps` steps (tokenize + fwd [+ bwd]) of workload `w` on `dev`;
+    returns the measurements (max over ranks of the timed region)."""
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_local_nb_b200 as nb
+    from block_sparse_local_nb_b200.dist import job_throughput, max_over_ranks, rank_seed
+    from block_sparse_local_nb_b200.inputs import make_attn_inputs
+
+    dt_code = nb.NB_BF16 if w.dtype == "bf16" else nb.NB_F32
+    B, H, N, D, R = w.batch, w.heads, w.n, w.d, w.R
+    stream = torch.cuda.Stream(device=dev)
+    base_seed = rank_seed(w.seed, rank)
+    q0, k0, v0, do0, lengths = make_attn_inputs(w, device=dev, seed=base_seed)
+    lengths_d = lengths.to(dev)
+    dna_np = dna_for_batch(w, seed=base_seed)
+    elem = q0.element_size()
+    ws_bytes = nb.attn_bwd_workspace_size(B, H, N, D, dt_code) if w.backward else 0
+    set_bytes = 8 * q0.numel() * elem + 2 * B * H * N * 4 + ws_bytes + 3 * dna_np.size
+    nsets = args.sets if args.sets > 0 else max(1, min(8, math.ceil(3 * L2_BYTES / set_bytes) + 1))
+    sets = []
+    for s in range(nsets):
+        if s == 0:
+            q, k, v, do = q0, k0, v0, do0
+        else:
+            q, k, v, do, _ = make_attn_inputs(w, device=dev, seed=base_seed + s)
+        st = {"q": q, "k": k, "v": v, "do": do, "o": torch.empty_like(q),
+              "lse": torch.empty((B, H, N), dtype=torch.float32, device=dev),
+              "dna": torch.from_numpy(dna_np).to(dev),
+              "ids": torch.empty(dna_np.size - 5, dtype=torch.int16, device=dev),
+              "packed": torch.empty((dna_np.size + 3) // 4, dtype=torch.uint8, device=dev)}
+        if w.backward:
+            st.update(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                      ws=torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev))
+        sets.append(st)
+    torch.cuda.synchronize(dev)
+
+    sptr = stream.cuda_stream
+    fwd = nb.nb_attn_fwd_causal if w.causal else nb.nb_attn_fwd
+    bwd = nb.nb_attn_bwd_causal if w.causal else nb.nb_attn_bwd
+
+    def step(st, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        nb.nb_tokenize_kmer(st["dna"], st["dna"].numel(), st["ids"], st["packed"], 6, sptr)
+        if ev is not None:
+            ev[1].record(stream)
+        fwd(st["q"], st["k"], st["v"], st["o"], st["lse"], lengths_d, B, H, N, D, R, dt_code, sptr)
+        if ev is not None:
+            ev[2].record(stream)
+        if w.backward:
+            bwd(st["q"], st["k"], st["v"], st["o"], st["do"], st["lse"], lengths_d, st["dq"],
+                st["dk"], st["dv"], st["ws"], ws_bytes, B, H, N, D, R, dt_code, sptr)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[dev.index])
+        torch.cuda.synchronize(dev)
+
+    with torch.cuda.stream(stream):
+        for s in range(warmup):
+            step(sets[s % nsets])
+    barrier()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        barrier()
+        start.record(stream)
+        for s in range(steps):
+            step(sets[s % nsets], evs[s])
+        end.record(stream)
+        barrier()
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
+    alg = algorithmic(w, lengths.tolist())
+    res = {
+        "w": w, "alg": alg, "elapsed_ms": elapsed_ms, "steps": steps, "nsets": nsets,
+        "set_bytes": set_bytes, "dna_bases": int(dna_np.size),
+        "value": job_throughput(alg["tokens"], steps, world, elapsed_ms),
+        "calls_ms": {
+            "nb_tokenize_kmer": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
+            "nb_attn_fwd": statistics.mean(e[1].elapsed_time(e[2]) for e in evs),
+            "nb_attn_bwd": statistics.mean(e[2].elapsed_time(e[3]) for e in evs) if w.backward else 0.0,
+        },
+        "clocks": sampler.summary(),
+        "launches_per_step": 2 + (3 if w.backward else 0),
+    }
+    res["inputs"] = (sets[0]["q"], sets[0]["k"], sets[0]["v"], sets[0]["do"])
+    res["lengths"] = lengths.numpy()
+    res["dna"] = dna_np
+    if not with_e2e:
+        del sets
+        return res
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies timed
+    st = sets[0]
+    for extra in sets[1:]:
+        extra.clear()
+    torch.cuda.empty_cache()
+    host = {name: st[name].cpu().pin_memory() for name in ("q", "k", "v", "do")}
+    host["dna"] = torch.from_numpy(dna_np).pin_memory()
+    host["lengths"] = lengths.pin_memory()
+    out_names = ("o", "lse", "ids", "packed") + (("dq", "dk", "dv") if w.backward else ())
+    outs = {name: torch.empty_like(st[name], device="cpu").pin_memory() for name in out_names}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    e_steps = max(1, min(steps, 5))
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            for name in ("q", "k", "v", "do", "dna"):
+                st[name].copy_(host[name], non_blocking=True)
+            lengths_d.copy_(host["lengths"], non_blocking=True)
+            step(st)
+            for name, t in outs.items():
+                t.copy_(st[name], non_blocking=True)
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        e_start.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e_end.record(stream)
+        barrier()
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
+    res["e2e"] = {"value": job_throughput(alg["tokens"], e_steps, world, e2e_ms), "unit": "tokens/s",
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps}
+    del sets, host, outs
+    return res
+
+
+def attention_line(res, peaks, peak_kind, world):
+    """The JSON fields of one attention workload's measurement."""
+    w, alg = res["w"], res["alg"]
+    steps = res["steps"]
+    ms_step = res["elapsed_ms"] / steps
+    timed_s = res["elapsed_ms"] / 1e3
+    smax = res["clocks"].get("sm_max_mhz")
+    calls = {}
+    fwd_ms, bwd_ms, tok_ms = (res["calls_ms"][c] for c in ("nb_attn_fwd", "nb_attn_bwd", "nb_tokenize_kmer"))
+    calls["nb_attn_fwd"] = roofline(alg["fwd_bytes"], alg["fwd_flops"], fwd_ms, peaks, timed_s, w.dtype, smax)
+    if w.backward:
+        calls["nb_attn_bwd"] = roofline(alg["bwd_bytes"], alg["bwd_flops"], bwd_ms, peaks, timed_s,
+                                        w.dtype, smax)
+    calls["nb_tokenize_kmer"] = roofline(tokenizer_bytes(res["dna_bases"]), 0, tok_ms, peaks,
+                                         timed_s, "u8")
+    for name, ms in res["calls_ms"].items():
+        if name in calls:
+            calls[name]["ms"] = ms
+    dom = "nb_attn_bwd" if w.backward and bwd_ms >= fwd_ms else "nb_attn_fwd"
+    roof = dict(calls[dom])
+    roof.pop("ms", None)
+    roof["traffic"] = recorded_traffic(dom, w.name)
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'fallback'})"
+    step_bytes = alg["fwd_bytes"] + (alg["bwd_bytes"] if w.backward else 0) + tokenizer_bytes(res["dna_bases"])
+    step_flops = alg["fwd_flops"] + (alg["bwd_flops"] if w.backward else 0)
+    step_roof = roofline(step_bytes, step_flops, ms_step, peaks, timed_s, w.dtype, smax)
+    cfg = workload_config(w)
+    cfg.update({"tokens_per_step": alg["tokens"],
+                "parallelism": f"dp{world} (independent batches)",
+                "l2": f"{res['nsets']} rotating input sets of {res['set_bytes'] / 2**20:.0f} MiB each "
+                      f"(> {L2_BYTES >> 20} MiB L2 between reuses)"})
+    return {
+        "value": res["value"], "unit": "tokens/s", "ms_per_step": ms_step,
+        "dtype": w.dtype, "config": cfg, "roofline": roof,
+        "step_roofline": {"bytes": step_bytes, "flops": step_flops, "bound": step_roof["bound"],
+                          "frac": step_roof["frac"], "roofline_ms": step_roof["roofline_ms"]},
+        "calls": calls, "clocks": res["clocks"],
+        "gpu_launches": res["launches_per_step"] * steps,
+    }
+
+
+def time_tokenizer(args, dev, steps, warmup):
+    """The 2**28-byte k-mer tokenizer workload alone: bases/s and the fraction
+    of the HBM roofline (1 byte read + 2.25 bytes written per base)."""
     import torch
 
     import block_sparse_local_nb_b200 as nb
     from block_sparse_local_nb_b200.inputs import DNA_BYTES, make_dna
 
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
     dna = make_dna(DNA_BYTES)
     seq = torch.from_numpy(dna).to(dev)
     ids = torch.empty(DNA_BYTES - 5, dtype=torch.int16, device=dev)
     packed = torch.empty(DNA_BYTES // 4, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
     sptr = stream.cuda_stream
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         nb.nb_tokenize_kmer(seq, DNA_BYTES, ids, packed, 6, sptr)
     torch.cuda.synchronize(dev)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(0)
+    sampler = ClockSampler(dev.index)
     with sampler:
         start.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             nb.nb_tokenize_kmer(seq, DNA_BYTES, ids, packed, 6, sptr)
         end.record(stream)
         torch.cuda.synchronize(dev)
-    ms = start.elapsed_time(end) / args.steps
+    ms = start.elapsed_time(end) / steps
     peaks, peak_kind = load_peaks()
-    hbm = float(peaks["hbm_gbs"])
-    alg_bytes = DNA_BYTES + 2 * (DNA_BYTES - 5) + DNA_BYTES // 4
-    achieved = alg_bytes / (ms / 1e3) / 1e9
-    line = {
+    roof = roofline(tokenizer_bytes(DNA_BYTES), 0, ms, peaks, ms * steps / 1e3, "u8")
+    roof.update(traffic=recorded_traffic("tokenize_kmer_kernel", "dna_2p28"),
+                kernel="tokenize_kmer_kernel", peak_source=peak_kind)
+    out = {
         "metric": "k-mer tokenizer bases/s and % of HBM roofline", "value": DNA_BYTES / (ms / 1e3),
-        "unit": "bases/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u8", "data": "synthetic",
+        "unit": "bases/s", "ms_per_step": ms, "steps": steps, "dtype": "u8",
         "config": {"workload": "dna_2p28", "bytes": DNA_BYTES, "k": 6, "n_fraction": 0.01,
                    "l2": "inputs and outputs (872 MB) larger than the 126 MB L2"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": recorded_traffic("tokenize_kmer_kernel", "dna_2p28"),
-                     "kernel": "tokenize_kmer_kernel", "peak_source": peak_kind},
-        "gpu_launches": args.steps, "clocks": sampler.summary(),
+        "roofline": roof, "gpu_launches": steps, "clocks": sampler.summary(),
     }
+    del seq, ids, packed
+    torch.cuda.empty_cache()
     if not args.no_cpu_baseline:
-        from threadpoolctl import threadpool_info
-
         from oracle import kmer_ids, pack_2bit
 
         sample = dna[: 1 << 24]
@@ -329,10 +577,10 @@ def run_tokenizer_workload(args):
         kmer_ids(sample, 6)
         pack_2bit(sample)
         dt = time.perf_counter() - t0
-        line["cpu_baseline"] = {"value": sample.size / dt, "unit": "bases/s", "cores": 1,
-                                "kind": "oracle", "sample": "first 2**24 bytes of the workload "
-                                "through the NumPy oracle (ids + packed stream)"}
-    print(json.dumps(line), flush=True)
+        out["cpu_baseline"] = {"value": sample.size / dt, "unit": "bases/s", "cores": 1,
+                               "kind": "oracle", "sample": "first 2**24 bytes of the workload "
+                               "through the NumPy oracle (ids + packed stream)"}
+    return out
 
 
 def run_batch_ids_workload(args):
@@ -350,7 +598,7 @@ def run_batch_ids_workload(args):
     blob, offsets = make_dna_batch()
     batch = offsets.size - 1
     windows = np.maximum(np.diff(offsets) - 5, 0)
-    n_pad = int(-(-windows.max() // 32) * 32)
+    n_pad = nb.nb_batch_ceiling(offsets, batch, 6)
     seqs = torch.from_numpy(blob).to(dev)
     off = torch.from_numpy(offsets).to(dev)
     ids = torch.empty((batch, n_pad), dtype=torch.int64, device=dev)
@@ -371,9 +619,10 @@ def run_batch_ids_workload(args):
         torch.cuda.synchronize(dev)
     ms = start.elapsed_time(end) / args.steps
     peaks, peak_kind = load_peaks()
-    hbm = float(peaks["hbm_gbs"])
     alg_bytes = blob.size + 8 * offsets.size + 8 * batch * n_pad + 4 * batch
-    achieved = alg_bytes / (ms / 1e3) / 1e9
+    roof = roofline(alg_bytes, 0, ms, peaks, ms * args.steps / 1e3, "u8")
+    roof.update(traffic=recorded_traffic("tokenize_batch_kernel", "dna_batch_ids"),
+                kernel="tokenize_batch_kernel", peak_source=peak_kind)
     line = {
         "metric": "batch tokenizer to model IDs windows/s and % of HBM roofline",
         "value": float(windows.sum()) / (ms / 1e3), "unit": "windows/s", "n_gpus": 1,
@@ -382,11 +631,7 @@ def run_batch_ids_workload(args):
         "config": {"workload": "dna_batch_ids", "sequences": int(batch), "bases": int(blob.size),
                    "n_pad": n_pad, "k": 6, "n_fraction": 0.01,
                    "l2": f"output ({8 * batch * n_pad / 2**20:.0f} MiB) larger than the 126 MB L2"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm,
-                     "traffic": recorded_traffic("tokenize_batch_kernel", "dna_batch_ids"),
-                     "kernel": "tokenize_batch_kernel", "peak_source": peak_kind},
-        "gpu_launches": args.steps, "clocks": sampler.summary(),
+        "roofline": roof, "gpu_launches": args.steps, "clocks": sampler.summary(),
     }
     if not args.no_cpu_baseline:
         from oracle.tokenizer import model_ids_batch
@@ -406,30 +651,39 @@ def run_batch_ids_workload(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="bf16_varlen")
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--sets", type=int, default=0, help="rotating input sets (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub", action="store_true", help="headline workload only")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
     from block_sparse_local_nb_b200.inputs import WORKLOADS
 
-    if args.workload == "dna_2p28":
-        if args.impl == "native" and int(os.environ.get("RANK", "0")) == 0:
-            run_tokenizer_workload(args)
-        return
-    if args.workload == "dna_batch_ids":
-        if args.impl == "native" and int(os.environ.get("RANK", "0")) == 0:
-            run_batch_ids_workload(args)
-        return
-    w = WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.workload == "dna_batch_ids":
+        if args.impl == "native" and rank == 0:
+            run_batch_ids_workload(args)
+        return
+    if args.workload == "dna_2p28":
+        if args.impl == "native" and rank == 0:
+            import torch
+
+            dev = torch.device("cuda", 0)
+            torch.cuda.set_device(dev)
+            line = time_tokenizer(args, dev, args.steps, args.warmup)
+            line.update(n_gpus=1, warmup=args.warmup, higher_is_better=True, scaling="weak",
+                        vs_baseline=None, data="synthetic")
+            print(json.dumps(line), flush=True)
+        return
+    w = WORKLOADS[args.workload]
 
     if args.impl == "reference":
         if rank == 0:
@@ -439,136 +693,14 @@ def main():
     import torch
     import torch.distributed as dist
 
-    import block_sparse_local_nb_b200 as nb
-    from block_sparse_local_nb_b200.dist import job_throughput, max_over_ranks, rank_seed
-    from block_sparse_local_nb_b200.inputs import make_attn_inputs
-
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
         import datetime
 
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    dt_code = nb.NB_BF16 if w.dtype == "bf16" else nb.NB_F32
-    B, H, N, D, R = w.batch, w.heads, w.n, w.d, w.R
-    stream = torch.cuda.Stream(device=dev)
-
-    # ---- resident inputs: rotating sets so each step's reads miss L2
-    per_set = None
-    sets = []
-    base_seed = rank_seed(w.seed, rank)
-    nsets = args.sets
-    q0, k0, v0, do0, lengths = make_attn_inputs(w, device=dev, seed=base_seed)
-    lengths_d = lengths.to(dev)
-    dna_np = dna_for_batch(w, seed=base_seed)
-    elem = q0.element_size()
-    set_bytes = (8 * q0.numel() * elem + 2 * B * H * N * 4
-                 + nb.attn_bwd_workspace_size(B, H, N, D, dt_code) + 3 * dna_np.size)
-    if nsets <= 0:
-        nsets = max(1, min(8, math.ceil(3 * L2_BYTES / set_bytes) + 1))
-    for s in range(nsets):
-        if s == 0:
-            q, k, v, do = q0, k0, v0, do0
-        else:
-            q, k, v, do, _ = make_attn_inputs(w, device=dev, seed=base_seed + s)
-        st = {"q": q, "k": k, "v": v, "do": do,
-              "o": torch.empty_like(q), "lse": torch.empty((B, H, N), dtype=torch.float32, device=dev),
-              "dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
-              "dna": torch.from_numpy(dna_np).to(dev),
-              "ids": torch.empty(dna_np.size - 5, dtype=torch.int16, device=dev),
-              "packed": torch.empty((dna_np.size + 3) // 4, dtype=torch.uint8, device=dev)}
-        ws_bytes = nb.attn_bwd_workspace_size(B, H, N, D, dt_code)
-        st["ws"] = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-        st["ws_bytes"] = ws_bytes
-        sets.append(st)
-    torch.cuda.synchronize(dev)
-
-    sptr = stream.cuda_stream
-    fwd = nb.nb_attn_fwd_causal if w.causal else nb.nb_attn_fwd
-    bwd = nb.nb_attn_bwd_causal if w.causal else nb.nb_attn_bwd
-
-    def step(st, ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        nb.nb_tokenize_kmer(st["dna"], st["dna"].numel(), st["ids"], st["packed"], 6, sptr)
-        if ev is not None:
-            ev[1].record(stream)
-        fwd(st["q"], st["k"], st["v"], st["o"], st["lse"], lengths_d, B, H, N, D, R, dt_code, sptr)
-        if ev is not None:
-            ev[2].record(stream)
-        if w.backward:
-            bwd(st["q"], st["k"], st["v"], st["o"], st["do"], st["lse"], lengths_d, st["dq"],
-                st["dk"], st["dv"], st["ws"], st["ws_bytes"], B, H, N, D, R, dt_code, sptr)
-        if ev is not None:
-            ev[3].record(stream)
-
-    launches_per_step = 1 + 1 + (3 if w.backward else 0)
-
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local_rank])
-        torch.cuda.synchronize(dev)
-
-    with torch.cuda.stream(stream):
-        for s in range(args.warmup):
-            step(sets[s % nsets])
-    barrier()
-
-    # ---- timed region: exactly K steps, per-call events on the launching stream
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local_rank)
-    with sampler:
-        barrier()
-        start.record(stream)
-        for s in range(args.steps):
-            step(sets[s % nsets], evs[s])
-        end.record(stream)
-        barrier()
-    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
-    tok_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
-
-    alg = algorithmic(w, lengths.tolist())
-    tokens_step = alg["tokens"]
-    value = job_throughput(tokens_step, args.steps, world, elapsed_ms)
-
-    # ---- end to end through the C ABI with host buffers (pinned), copies timed
-    host = {}
-    for name in ("q", "k", "v", "do"):
-        host[name] = sets[0][name].cpu().pin_memory()
-    host["dna"] = torch.from_numpy(dna_np).pin_memory()
-    host["lengths"] = lengths.pin_memory()
-    outs = {name: torch.empty_like(sets[0][name], device="cpu").pin_memory()
-            for name in ("o", "lse", "dq", "dk", "dv", "ids", "packed")}
-    st = sets[0]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs.values())
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        def e2e_step():
-            for name in ("q", "k", "v", "do", "dna"):
-                st[name].copy_(host[name], non_blocking=True)
-            lengths_d.copy_(host["lengths"], non_blocking=True)
-            step(st)
-            for name, t in outs.items():
-                t.copy_(st[name], non_blocking=True)
-        for _ in range(3):
-            e2e_step()
-        barrier()
-        e_start.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e_end.record(stream)
-        barrier()
-    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
-    e2e_value = job_throughput(tokens_step, args.steps, world, e2e_ms)
-
+    res = time_attention(w, args, dev, rank, world, True, args.steps, args.warmup)
     if world > 1:
         dist.barrier(device_ids=[local_rank])
         dist.destroy_process_group()
@@ -576,56 +708,34 @@ def main():
         return
 
     peaks, peak_kind = load_peaks()
-    hbm = float(peaks["hbm_gbs"])
-    bf16 = float(peaks["bf16_tflops"])
-    fwd_avg = statistics.mean(fwd_ms)
-    bwd_avg = statistics.mean(bwd_ms) if w.backward else 0.0
-    tok_avg = statistics.mean(tok_ms)
-    # dominant call of the step
-    if w.backward and bwd_avg >= fwd_avg:
-        dom, dom_ms, dom_bytes, dom_flops = "nb_attn_bwd", bwd_avg, alg["bwd_bytes"], alg["bwd_flops"]
-    else:
-        dom, dom_ms, dom_bytes, dom_flops = "nb_attn_fwd", fwd_avg, alg["fwd_bytes"], alg["fwd_flops"]
-    t_hbm = dom_bytes / (hbm * 1e9)
-    t_tc = dom_flops / (bf16 * 1e12)
-    if t_hbm >= t_tc:
-        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s"}
-    else:
-        achieved = dom_flops / (dom_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic(dom, w.name)
-    roof["kernel"] = dom
-    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'fallback'})"
-
-    step_bytes = alg["fwd_bytes"] + (alg["bwd_bytes"] if w.backward else 0)
-    step_flops = alg["fwd_flops"] + (alg["bwd_flops"] if w.backward else 0)
-    ms_per_step = elapsed_ms / args.steps
+    body = attention_line(res, peaks, peak_kind, world)
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "metric": METRIC, "value": body["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": body["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
-        "data": "synthetic",
-        "config": {"workload": w.name, "desc": w.desc + " + k=6 tokenization of the batch's "
-                   f"{B}x({N}+5) bases", "batch": B, "heads": H, "n": N, "d": D, "R": R,
-                   "tokens_per_step": tokens_step, "parallelism": f"dp{world} (independent batches)",
-                   "l2": f"{nsets} rotating input sets of {set_bytes / 2**20:.0f} MiB each "
-                         f"(> {L2_BYTES >> 20} MiB L2 between reuses)"},
-        "roofline": roof,
-        "step_roofline": {"bytes": step_bytes, "flops": step_flops,
-                          "hbm_frac": step_bytes / (ms_per_step / 1e3) / (hbm * 1e9),
-                          "tensor_frac": step_flops / (ms_per_step / 1e3) / (bf16 * 1e12),
-                          "frac_of_roofline": max(step_bytes / (hbm * 1e9), step_flops / (bf16 * 1e12))
-                          / (ms_per_step / 1e3)},
-        "calls_ms": {"nb_tokenize_kmer": tok_avg, "nb_attn_fwd": fwd_avg, "nb_attn_bwd": bwd_avg},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": sampler.summary(),
+        "data": "synthetic", "config": body["config"], "roofline": body["roofline"],
+        "step_roofline": body["step_roofline"], "calls": body["calls"], "e2e": res["e2e"],
+        "gpu_launches": body["gpu_launches"], "clocks": body["clocks"],
     }
+    if world == 1 and not args.no_sub:
+        subs = {}
+        for name in SUB_WORKLOADS:
+            if name == args.workload:
+                continue
+            if name == "dna_2p28":
+                subs[name] = time_tokenizer(args, dev, max(args.steps, 20), args.warmup)
+                continue
+            sw = WORKLOADS[name]
+            sres = time_attention(sw, args, dev, 0, 1, False, max(args.steps, 20), args.warmup)
+            sres.pop("inputs")
+            torch.cuda.empty_cache()
+            sub = attention_line(sres, peaks, peak_kind, 1)
+            sub["metric"] = METRIC
+            subs[name] = sub
+        line["sub_results"] = subs
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"] = cpu_baseline(w, window_fetcher(res["inputs"]), res["lengths"],
+                                            res["dna"])
     print(json.dumps(line), flush=True)
 
 

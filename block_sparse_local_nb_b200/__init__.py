@@ -16,6 +16,7 @@ from .binding import (  # noqa: F401
     nb_attn_bwd_causal,
     nb_attn_fwd,
     nb_attn_fwd_causal,
+    nb_batch_ceiling,
     nb_kernel_error,
     nb_status_string,
     nb_tokenize_batch,

@@ -35,6 +35,7 @@ _SIGS = [
                                 _I, _I, _I, _I, _I, _I, _P]),
     ("nb_tokenize_kmer", _I, [_P, ctypes.c_int64, _P, _P, _I, _P]),
     ("nb_tokenize_batch", _I, [_P, _P, _I, _I, _P, _P, _I, _P]),
+    ("nb_batch_ceiling", _I, [_P, _I, _I, ctypes.POINTER(ctypes.c_int32)]),
 ]
 
 
@@ -151,3 +152,17 @@ def nb_tokenize_batch(seqs, offsets, batch, k, input_ids, lengths, n_pad, stream
     if check:
         _check(st, "nb_tokenize_batch")
     return st
+
+
+def nb_batch_ceiling(offsets, batch, k=6) -> int:
+    """The dynamic ceiling (n_pad) of a batch from its HOST int64 offsets
+    [batch + 1] (a NumPy array or a sequence of ints)."""
+    import numpy as np
+
+    off = np.ascontiguousarray(np.asarray(offsets, dtype=np.int64))
+    if off.size < batch + 1:
+        raise ValueError("offsets must hold batch + 1 entries")
+    out = ctypes.c_int32(0)
+    st = lib().nb_batch_ceiling(off.ctypes.data if off.size else None, batch, k, ctypes.byref(out))
+    _check(st, "nb_batch_ceiling")
+    return int(out.value)

@@ -104,6 +104,18 @@ nb_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* 
   return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
 }
 
+// Pointer checks of the backward (null -> invalid, alignment).
+nb_status bwd_pointers(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, const int32_t* lengths, void* dq,
+                       void* dk, void* dv) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return NB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (lengths && (reinterpret_cast<uintptr_t>(lengths) & 3u)))
+    return NB_ERR_MISALIGNED;
+  return NB_OK;
+}
+
 nb_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                    const float* lse, const int32_t* lengths, void* dq, void* dk, void* dv,
                    void* workspace, size_t workspace_bytes, int batch, int heads, int n, int d,
@@ -112,11 +124,8 @@ nb_status attn_bwd(const void* q, const void* k, const void* v, const void* o, c
   if (st != NB_OK) return st;
   if (static_cast<int64_t>(batch) * heads * n == 0) return NB_OK;
   if (dtype != NB_BF16) return NB_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return NB_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
-      (lengths && (reinterpret_cast<uintptr_t>(lengths) & 3u)))
-    return NB_ERR_MISALIGNED;
+  st = bwd_pointers(q, k, v, o, dout, lse, lengths, dq, dk, dv);
+  if (st != NB_OK) return st;
   const int64_t rows = static_cast<int64_t>(batch) * heads * n;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
       workspace_bytes < nb::bwd_workspace_bytes(rows, d))
@@ -130,6 +139,25 @@ nb_status attn_bwd(const void* q, const void* k, const void* v, const void* o, c
 }
 
 }  // namespace
+
+namespace nb {
+
+nb_status bwd_host_checks(int batch, int heads, int n, int d, int R, int dtype) {
+  const nb_status st = check_shape(batch, heads, n, d, R, dtype);
+  if (st != NB_OK) return st;
+  if (static_cast<int64_t>(batch) * heads * n == 0) return NB_OK;
+  return dtype == NB_BF16 ? NB_OK : NB_ERR_UNSUPPORTED;
+}
+
+nb_status bwd_pointer_checks(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, const int32_t* lengths,
+                             void* dq, void* dk, void* dv) {
+  return bwd_pointers(q, k, v, o, dout, lse, lengths, dq, dk, dv);
+}
+
+nb_status device_check() { return check_device(); }
+
+}  // namespace nb
 
 extern "C" {
 
@@ -225,6 +253,21 @@ nb_status nb_tokenize_batch(const uint8_t* seqs, const int64_t* offsets, int bat
   cudaError_t e = nb::launch_tokenize_batch(seqs, offsets, batch, k, input_ids, lengths, n_pad,
                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
+}
+
+nb_status nb_batch_ceiling(const int64_t* offsets, int batch, int k, int32_t* n_pad) {
+  if (!n_pad || batch < 0 || (batch > 0 && !offsets)) return NB_ERR_INVALID_ARG;
+  if (k < 1 || k > 7) return NB_ERR_UNSUPPORTED;
+  int64_t windows = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t bases = offsets[b + 1] - offsets[b];
+    const int64_t w = bases >= k ? bases - k + 1 : 0;
+    if (w > windows) windows = w;
+  }
+  const int64_t ceil32 = (windows + NB_BLOCK - 1) / NB_BLOCK * NB_BLOCK;
+  if (ceil32 > INT32_MAX) return NB_ERR_INVALID_ARG;
+  *n_pad = static_cast<int32_t>(ceil32);
+  return NB_OK;
 }
 
 }  // extern "C"

@@ -11,7 +11,7 @@
 #include <math.h>
 
 #include "nb_internal.h"
-#include "warp_mma.cuh"
+#include "sm100.cuh"
 
 namespace nb {
 namespace {

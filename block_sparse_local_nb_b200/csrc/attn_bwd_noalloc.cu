@@ -20,11 +20,17 @@
 // threads) race on it and must be serialised by the caller.  The kernels
 // rewrite every byte they read from it on each call (the row term and the
 // zeroed dQ accumulator), so contents left by an earlier call do not matter.
+//
+// The checks run in this order, all on the host before the symbol lookup, so
+// a rejected call neither launches nor loads the array: shape and dtype (as
+// nb_attn_bwd), the scratch limit (NB_ERR_WORKSPACE), pointers (as
+// nb_attn_bwd), the device (NB_ERR_DEVICE).
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "../../include/nb.h"
+#include "nb_internal.h"
 
 namespace {
 
@@ -44,7 +50,7 @@ nb_status scratch_address(void** out) {
   if (g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();  // consume the error so an unrelated later call does not report it
+      cudaGetLastError();  // the failed lookup's error, so an unrelated later call does not report it
       return NB_ERR_CUDA;
     }
     g_scratch_addr[dev] = p;
@@ -60,13 +66,17 @@ extern "C" NB_API nb_status nb_attn_bwd_noalloc(const void* q, const void* k, co
                                                 const int32_t* lengths, void* dq, void* dk,
                                                 void* dv, int batch, int heads, int n, int d,
                                                 int R, int dtype, void* stream) {
+  nb_status st = nb::bwd_host_checks(batch, heads, n, d, R, dtype);
+  if (st != NB_OK) return st;
   const size_t need = nb_attn_bwd_workspace_size(batch, heads, n, d, dtype);
-  if (need == 0)  // empty or invalid problem: nb_attn_bwd returns its status without launching
-    return nb_attn_bwd(q, k, v, o, dout, lse, lengths, dq, dk, dv, nullptr, 0, batch, heads, n,
-                       d, R, dtype, stream);
+  if (need == 0) return NB_OK;                      // empty problem: nothing to do
   if (need > kScratchBytes) return NB_ERR_WORKSPACE;  // beyond the built-in scratch
+  st = nb::bwd_pointer_checks(q, k, v, o, dout, lse, lengths, dq, dk, dv);
+  if (st != NB_OK) return st;
+  st = nb::device_check();
+  if (st != NB_OK) return st;
   void* scratch = nullptr;
-  const nb_status st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != NB_OK) return st;
   return nb_attn_bwd(q, k, v, o, dout, lse, lengths, dq, dk, dv, scratch, kScratchBytes, batch,
                      heads, n, d, R, dtype, stream);

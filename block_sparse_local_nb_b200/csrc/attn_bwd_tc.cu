@@ -34,7 +34,6 @@
 #include "nb_internal.h"
 #include "schedule.cuh"
 #include "sm100.cuh"
-#include "warp_mma.cuh"
 
 namespace nb {
 namespace {

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/nb.h"
+
 namespace nb {
 
 constexpr int kBlock = 32;  // band block size B (NucleoByte page, section 3)
@@ -84,6 +86,13 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
+
+// Host-side argument checks of the C ABI, shared by its entry points (api.cu).
+nb_status bwd_host_checks(int batch, int heads, int n, int d, int R, int dtype);  // shape, dtype
+nb_status bwd_pointer_checks(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, const int32_t* lengths,
+                             void* dq, void* dk, void* dv);  // null pointers, alignment
+nb_status device_check();  // the current device is an sm_100 GPU
 
 cudaError_t launch_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
                                  int k, cudaStream_t stream);

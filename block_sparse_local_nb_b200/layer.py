@@ -28,15 +28,14 @@ PAD_ID = 0
 
 def ceiling_layout(base_counts: Sequence[int], k: int = 6) -> tuple[np.ndarray, int]:
     """Offsets (int64 [batch + 1]) of the concatenated sequences and the
-    dynamic ceiling n_pad for sequences of the given base counts."""
+    dynamic ceiling n_pad (computed by the library's nb_batch_ceiling) for
+    sequences of the given base counts."""
     counts = np.asarray([int(c) for c in base_counts], dtype=np.int64)
     if (counts < 0).any():
         raise ValueError("base counts must be non-negative")
     offsets = np.zeros(counts.size + 1, dtype=np.int64)
     np.cumsum(counts, out=offsets[1:])
-    windows = int(np.maximum(counts - k + 1, 0).max()) if counts.size else 0
-    n_pad = -(-windows // BLOCK) * BLOCK
-    return offsets, n_pad
+    return offsets, nb.nb_batch_ceiling(offsets, counts.size, k)
 
 
 def collate(seqs: Sequence[bytes], k: int = 6, device=None, stream=None):

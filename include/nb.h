@@ -18,10 +18,16 @@
  *
  * Conventions shared by every call:
  *   - Every pointer argument is a DEVICE pointer unless stated otherwise.  The
- *     caller owns every buffer; the library allocates no device memory and
+ *     caller owns every buffer; no call allocates device memory.  The library
  *     keeps no state between calls except per-device caches (device
- *     properties, symbol addresses) and the kernel error word read by
- *     nb_kernel_error.
+ *     properties, the device addresses of its two __device__ variables) and
+ *     those variables: the kernel error word read by nb_kernel_error (4 bytes)
+ *     and the fixed scratch array of nb_attn_bwd_noalloc
+ *     (NB_NOALLOC_SCRATCH_BYTES = 64 MiB), which loading the library's device
+ *     code reserves on every GPU it runs on, until the process exits.  The
+ *     address caches assume the device's primary context lives as long as
+ *     the process: resetting a device (cudaDeviceReset) after a call of this
+ *     library on it is not supported.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream).  Arguments are validated on the host first: an invalid
  *     call returns a negative nb_status and launches nothing.  A failed launch
@@ -220,6 +226,21 @@ NB_API nb_status nb_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids
 #define NB_PAD_ID 0
 NB_API nb_status nb_tokenize_batch(const uint8_t* seqs, const int64_t* offsets, int batch, int k,
                                    int64_t* input_ids, int32_t* lengths, int n_pad, void* stream);
+
+/*
+ * nb_batch_ceiling - the dynamic ceiling of a batch for nb_tokenize_batch: the
+ * smallest multiple of 32 that holds the longest sequence's k-mer windows.
+ * (NucleoByte page, section 2 item 2 "Dynamic Ceiling Hardware Alignment": a
+ * batch is padded only up to the next multiple of 32 above its longest
+ * sequence, not to a fixed maximum length.)
+ * offsets in : HOST int64 [batch + 1], the same offsets nb_tokenize_batch takes;
+ *              sequence b has max(0, offsets[b+1] - offsets[b]) bases and
+ *              max(0, bases - k + 1) windows.
+ * n_pad   out: HOST int32; 0 for an empty batch or one without a window.
+ * k: 1..7.  batch >= 0.  A ceiling above INT32_MAX returns NB_ERR_INVALID_ARG.
+ * Runs on the host only (no device, no stream, no launch).
+ */
+NB_API nb_status nb_batch_ceiling(const int64_t* offsets, int batch, int k, int32_t* n_pad);
 
 #ifdef __cplusplus
 }

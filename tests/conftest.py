@@ -16,6 +16,20 @@ def pytest_configure(config):
 
 
 @pytest.fixture(scope="session")
+def built_lib():
+    """The C-ABI library, built in-tree first when it is missing (host-only
+    entry points of it run without a GPU)."""
+    lib_path = os.path.join(ROOT, "block_sparse_local_nb_b200", "libnb_b200.so")
+    if not os.path.exists(lib_path):
+        from block_sparse_local_nb_b200.build import build
+
+        build()
+    from block_sparse_local_nb_b200 import binding
+
+    return binding.lib()
+
+
+@pytest.fixture(scope="session")
 def golden_dir():
     return GOLDEN
 

@@ -180,3 +180,20 @@ def test_causal_entry_points_validate_like_the_band(lib, kw, status):
 def test_causal_backward_rejects_fp32(lib):
     assert lib.nb_attn_bwd_causal(16, 16, 16, 16, 16, 16, None, 16, 16, 16, 256, 1 << 30, 1, 1, 64,
                                   64, 1, F32, None) == NB_ERR_UNSUPPORTED
+
+
+def test_noalloc_rejects_on_the_host(lib):
+    """nb_attn_bwd_noalloc checks shape, dtype, its scratch limit and pointers
+    before it touches the device: these calls return without a GPU."""
+    fn = lib.nb_attn_bwd_noalloc
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p] * 10 + [ctypes.c_int] * 6 + [ctypes.c_void_p]
+    nulls = [None] * 10
+    # 1 x 8 x 65536 x 64 needs about 130 MiB of scratch, beyond the 64 MiB array
+    assert fn(*nulls, 1, 8, 65536, 64, 1, BF16, None) == NB_ERR_WORKSPACE
+    assert fn(*nulls, 1, 1, 64, 64, 1, F32, None) == NB_ERR_UNSUPPORTED
+    assert fn(*nulls, 1, 1, 48, 64, 1, BF16, None) == NB_ERR_INVALID_ARG
+    assert fn(*nulls, 1, 1, 64, 64, 1, BF16, None) == NB_ERR_INVALID_ARG  # null pointers
+    assert fn(*nulls, 0, 1, 64, 64, 1, BF16, None) == NB_OK  # empty problem
+    ptrs = [16] * 6 + [None] + [16, 16, 24]  # dv not 16-byte aligned
+    assert fn(*ptrs, 1, 1, 64, 64, 1, BF16, None) == NB_ERR_MISALIGNED

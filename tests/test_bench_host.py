@@ -45,3 +45,30 @@ def test_peaks_are_read_or_fall_back():
     peaks, kind = bench.load_peaks()
     assert kind in ("measured", "fallback")
     assert float(peaks["hbm_gbs"]) > 0
+
+
+def test_oracle_windows_cover_valid_rows_only():
+    from block_sparse_local_nb_b200.inputs import WORKLOADS
+
+    w = WORKLOADS["bf16_n1m"]
+    nb = w.n // 32
+    for step in range(50):
+        b, h, lo, hi = bench.oracle_window(w, [w.n], step)
+        assert 0 <= lo < hi <= nb and hi - lo == 256 and 0 <= h < w.heads and b == 0
+    w = WORKLOADS["bf16_varlen"]
+    lengths = [1030, 4096, 2000, 1]
+    for step in range(20):
+        b, h, lo, hi = bench.oracle_window(w, lengths, step)
+        assert (lo, hi) == (0, (lengths[b] + 31) // 32)
+
+
+def test_roofline_picks_the_slower_bound():
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 100.0, "bf16_tflops_sustained": 50.0}
+    r = bench.roofline(2e9, 1e12, 4.0, peaks, 0.1, "bf16")  # 2 ms of HBM vs 10 ms of tensor
+    assert r["bound"] == "tensor" and r["peak"] == 100.0 and r["peak_kind"] == "burst"
+    assert r["frac"] == pytest.approx(10.0 / 4.0) and r["roofline_ms"] == pytest.approx(10.0)
+    r = bench.roofline(2e9, 1e12, 40.0, peaks, 5.0, "bf16")  # a long timed region: sustained peak
+    assert r["peak"] == 50.0 and r["peak_kind"] == "sustained"
+    r = bench.roofline(8e9, 1e9, 16.0, peaks, 0.1, "bf16")  # 8 ms of HBM vs 0.01 ms of tensor
+    assert r["bound"] == "hbm" and r["frac"] == pytest.approx(0.5)
+    assert bench.tokenizer_bytes(10) == 10 + 2 * 5 + 3

@@ -220,19 +220,41 @@ def test_bf16_varlen_workload(name):
             assert (t[b, :, Lb:] == 0).all() or torch.isneginf(t[b, :, Lb:]).all()
 
 
+def _full_size_windows(w, width, seed):
+    """(head, first block) of the windows checked on a full-length, batch-1
+    workload: the first and last window and one random window of every head,
+    plus windows on the persistent kernels' last wave of work items (one
+    128-row tile per item, items handed round-robin to one CTA per SM): the
+    wave's first tile, its middle and the sequence's last tile, where each
+    CTA runs its final item and its deferred epilogue."""
+    nb = w.n // BLOCK
+    rng = np.random.default_rng(seed)
+    out = []
+    for h in range(w.heads):
+        out += [(h, 0), (h, nb - width), (h, int(rng.integers(0, nb - width)))]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    tiles = w.n // 128
+    items = w.heads * tiles
+    first_last = (items - 1) // sms * sms  # first item of the last wave
+    for it in (first_last, (first_last + items) // 2, items - 1):
+        h, tile = divmod(it, tiles)
+        lo = min(max(0, 4 * tile - width // 2), nb - width)
+        out.append((h, lo))
+    return out
+
+
 def test_bf16_n131k_workload():
-    """bf16, 1 x 16 x 131072 x 128, R = 4: sampled windows incl. both ends."""
+    """bf16, 1 x 16 x 131072 x 128, R = 4: first, last and a random window of
+    every head, and the persistent kernels' last wave."""
     w = WORKLOADS["bf16_n131k"]
     tensors, outs, lengths = _run_workload(w)
-    nb = w.n // BLOCK
-    rng = np.random.default_rng(1)
-    for h, lo in [(0, 0), (15, nb - 12), (7, 2000)] + [
-            (int(rng.integers(16)), int(rng.integers(0, nb - 12))) for _ in range(3)]:
+    for h, lo in _full_size_windows(w, 12, seed=1):
         _check_window(w, tensors, outs, (0, h), lo, lo + 12, lengths)
 
 
 def test_bf16_n1m_workload():
-    """bf16, 1 x 8 x 1048576 x 64, R = 8: sampled windows; peak memory linear in n."""
+    """bf16, 1 x 8 x 1048576 x 64, R = 8: first, last and a random window of
+    every head, and the persistent kernels' last wave; peak memory linear in n."""
     w = WORKLOADS["bf16_n1m"]
     torch.cuda.reset_peak_memory_stats()
     tensors, outs, lengths = _run_workload(w)
@@ -240,8 +262,5 @@ def test_bf16_n1m_workload():
     elems = w.batch * w.heads * w.n * w.d
     # 9 bf16 tensors (q k v do o dq dk dv + slack), lse, D and the fp32 dQ accumulator
     assert peak <= elems * 2 * 9 + elems * 4 + w.batch * w.heads * w.n * 8 + (64 << 20)
-    nb = w.n // BLOCK
-    rng = np.random.default_rng(2)
-    for h, lo in [(0, 0), (7, nb - 20)] + [
-            (int(rng.integers(8)), int(rng.integers(0, nb - 20))) for _ in range(3)]:
+    for h, lo in _full_size_windows(w, 20, seed=2):
         _check_window(w, tensors, outs, (0, h), lo, lo + 20, lengths)

@@ -51,13 +51,17 @@ def test_noalloc_matches_workspace_backward_on_consecutive_calls(d):
         want = run_bwd(q, k, v, o, do, lse, lengths, R)
         got = _call(fn, q, k, v, o, do, lse, lengths, R)
         torch.cuda.synchronize()
-        for name, g, w in zip(("dq", "dk", "dv"), got, want):
-            assert rel_fro(f64(g), f64(w)) <= GRAD_RFRO_BF16, name
+        # dK and dV are deterministic: bit-identical to the workspace path
+        assert torch.equal(got[1], want[1]) and torch.equal(got[2], want[2])
+        # dQ is accumulated with fp32 atomics (order may differ): within the bf16 bar
+        assert rel_fro(f64(got[0]), f64(want[0])) <= GRAD_RFRO_BF16
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     fn = _noalloc()
     batch, heads, n, d = 1, 8, 65536, 64  # needs about 130 MiB of scratch
     assert nb.attn_bwd_workspace_size(batch, heads, n, d, nb.NB_BF16) > SCRATCH_BYTES
-    st = fn(16, 16, 16, 16, 16, 16, None, 16, 16, 16, batch, heads, n, d, 1, nb.NB_BF16, None)
+    # every pointer null: whatever the order of the checks, the call fails on the host
+    st = fn(None, None, None, None, None, None, None, None, None, None, batch, heads, n, d, 1,
+            nb.NB_BF16, None)
     assert st == NB_ERR_WORKSPACE

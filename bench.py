@@ -658,6 +658,9 @@ def main():
     ap.add_argument("--sets", type=int, default=0, help="rotating input sets (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="headline workload only")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override n of a full-length workload (a smaller case of the same "
+                         "shape, e.g. for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -684,6 +687,13 @@ def main():
             print(json.dumps(line), flush=True)
         return
     w = WORKLOADS[args.workload]
+    if args.seq_len:
+        if w.varlen is not None or args.seq_len % 32:
+            ap.error("--seq-len applies to full-length workloads and must be a multiple of 32")
+        import dataclasses
+
+        w = dataclasses.replace(w, n=args.seq_len, name=f"{w.name}@n{args.seq_len}",
+                                desc=w.desc.replace(str(w.n), str(args.seq_len)))
 
     if args.impl == "reference":
         if rank == 0:

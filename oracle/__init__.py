@@ -24,5 +24,6 @@ from .attention import (  # noqa: F401
     attn_bwd_dense,
     attn_fwd_banded,
     attn_bwd_banded,
+    attn_bwd_from_saved,
 )
 from .tokenizer import kmer_ids, pack_2bit, N_FLAG_BASE  # noqa: F401

@@ -244,3 +244,54 @@ def attn_bwd_banded(q, k, v, do, R: int, lengths=None, causal: bool = False):
                 dq[b, h, r0:r0 + rows] = scale * (dS @ Kb)
                 dk[b, h, k0:k1] += scale * (dS.T @ Qi)
     return dq, dk, dv
+
+
+def attn_bwd_from_saved(q, k, v, o, do, lse, R: int, lengths=None, causal: bool = False):
+    """Analytic gradients from the forward's saved outputs, as the page's
+    backward uses them (NucleoByte page, section 3 "Custom Backpropagation"):
+    the probabilities are rebuilt from the stored log-sum-exp,
+    P_ij = exp(scale Q_i K_j^T - lse_i) over the band's visible keys, and the
+    row term is D_i = sum_k dO_ik O_ik with the given O.  With O and lse from
+    :func:`attn_fwd_banded` of the same inputs this is :func:`attn_bwd_banded`;
+    the difference is that a row's P and D come from the given lse and O, not
+    from the keys this call sees (a shard of a longer sequence sees only part
+    of a halo row's keys, while the row's lse and O are the whole sequence's).
+    Rows >= L_b and rows whose lse is -inf contribute nothing.
+    """
+    q, k, v, o, do = _f64(q), _f64(k), _f64(v), _f64(o), _f64(do)
+    lse = _f64(lse)
+    batch, heads, n, d = q.shape
+    if n % BLOCK:
+        raise ValueError("n must be a multiple of the block size")
+    nb = n // BLOCK
+    lens = _lengths(lengths, batch, n)
+    scale = 1.0 / math.sqrt(d)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(batch):
+        L = int(lens[b])
+        for i in range(nb):
+            r0 = i * BLOCK
+            rows = min(BLOCK, L - r0)
+            if rows <= 0:
+                break
+            j0, j1 = _band(i, R, nb, causal)
+            k0, k1 = j0 * BLOCK, min((j1 + 1) * BLOCK, L)
+            for h in range(heads):
+                Qi = q[b, h, r0:r0 + rows]
+                dOi = do[b, h, r0:r0 + rows]
+                Kb, Vb = k[b, h, k0:k1], v[b, h, k0:k1]
+                S = scale * (Qi @ Kb.T)
+                if causal:
+                    S = _causal_cut(S, r0, k0)
+                li = lse[b, h, r0:r0 + rows][:, None]
+                with np.errstate(invalid="ignore"):
+                    P = np.where(np.isfinite(li), np.exp(S - li), 0.0)
+                D = (dOi * o[b, h, r0:r0 + rows]).sum(axis=1)
+                dP = dOi @ Vb.T
+                dS = P * (dP - D[:, None])
+                dv[b, h, k0:k1] += P.T @ dOi
+                dq[b, h, r0:r0 + rows] = scale * (dS @ Kb)
+                dk[b, h, k0:k1] += scale * (dS.T @ Qi)
+    return dq, dk, dv

@@ -180,3 +180,43 @@ def test_causal_mutation_is_caught(name, old, new):
     except ValueError:  # the mutant cannot even evaluate the pins (an empty band)
         caught = True
     assert caught, name
+
+
+def _saved_pin_fails(mod):
+    """The backward from saved outputs: equal to the unmutated plain backward
+    when O and lse come from the forward, and a row's lse raised by ln 2
+    halves that row's P (so its dV contribution)."""
+    rng = np.random.default_rng(7)
+    for causal in (False, True):
+        q, k, v, do = (rng.standard_normal((1, 2, 128, 4)) for _ in range(4))
+        o, lse = att.attn_fwd_banded(q, k, v, 1, [100], causal=causal)
+        want = att.attn_bwd_banded(q, k, v, do, 1, [100], causal=causal)
+        got = mod.attn_bwd_from_saved(q, k, v, o, do, lse, 1, [100], causal=causal)
+        if not all(np.allclose(g, w, atol=1e-10) for g, w in zip(got, want)):
+            return True
+    q, k, v, do = (rng.standard_normal((1, 1, 64, 4)) for _ in range(4))
+    o, lse = att.attn_fwd_banded(q, k, v, 0)
+    do[0, 0, 32:] = 0
+    lse2 = lse.copy()
+    lse2[0, 0, :32] += math.log(2.0)
+    dv1 = mod.attn_bwd_from_saved(q, k, v, o, do, lse, 0)[2]
+    dv2 = mod.attn_bwd_from_saved(q, k, v, o, do, lse2, 0)[2]
+    return not np.allclose(dv2, dv1 / 2, atol=1e-12)
+
+
+SAVED_MUTATIONS = [
+    ("saved backward renormalises instead of using lse",
+     "P = np.where(np.isfinite(li), np.exp(S - li), 0.0)",
+     "P = np.where(np.isfinite(li), _softmax_rows(S)[0], 0.0)"),
+    ("saved backward row term from dO only", "D = (dOi * o[b, h, r0:r0 + rows]).sum(axis=1)",
+     "D = (dOi * dOi).sum(axis=1)"),
+    ("saved backward drops the scale of lse", "np.exp(S - li)", "np.exp(S / scale - li)"),
+]
+
+
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")
+@pytest.mark.parametrize("name,old,new", SAVED_MUTATIONS, ids=[m[0] for m in SAVED_MUTATIONS])
+def test_saved_backward_mutation_is_caught(name, old, new):
+    assert SRC_ATT.count(old) == 1, name
+    mod = _load_mutant(SRC_ATT.replace(old, new), "mutant_saved")
+    assert _saved_pin_fails(mod), name

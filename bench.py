@@ -342,6 +342,14 @@ def cpu_baseline(w, fetch, lengths, dna, budget_s=10.0):
                       f"has {os.cpu_count()} logical cores"}
 
 
+def check_kernel_error(nb):
+    """A kernel that gave up on a bounded wait leaves a code in the library's
+    error word; a timing that includes such a launch is not a measurement."""
+    code = nb.nb_kernel_error(clear=True)
+    if code:
+        raise RuntimeError(f"a kernel recorded wait-timeout code {code:#x}: no valid timing")
+
+
 def workload_config(w):
     return {"workload": w.name, "desc": w.desc + " + k=6 tokenization of the batch's "
             f"{w.batch}x({w.n}+5) bases", "batch": w.batch, "heads": w.heads, "n": w.n,
@@ -429,6 +437,7 @@ def time_attention(w, args, dev, rank, world, with_e2e, steps, warmup):
         end.record(stream)
         barrier()
     elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
+    check_kernel_error(nb)
     alg = algorithmic(w, lengths.tolist())
     res = {
         "w": w, "alg": alg, "elapsed_ms": elapsed_ms, "steps": steps, "nsets": nsets,
@@ -481,6 +490,7 @@ def time_attention(w, args, dev, rank, world, with_e2e, steps, warmup):
         e_end.record(stream)
         barrier()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
+    check_kernel_error(nb)
     res["e2e"] = {"value": job_throughput(alg["tokens"], e_steps, world, e2e_ms), "unit": "tokens/s",
                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps}
     del sets, host, outs
@@ -555,6 +565,7 @@ def time_tokenizer(args, dev, steps, warmup):
             nb.nb_tokenize_kmer(seq, DNA_BYTES, ids, packed, 6, sptr)
         end.record(stream)
         torch.cuda.synchronize(dev)
+    check_kernel_error(nb)
     ms = start.elapsed_time(end) / steps
     peaks, peak_kind = load_peaks()
     roof = roofline(tokenizer_bytes(DNA_BYTES), 0, ms, peaks, ms * steps / 1e3, "u8")
@@ -658,6 +669,8 @@ def main():
     ap.add_argument("--sets", type=int, default=0, help="rotating input sets (0 = auto)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="headline workload only")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffers) measurement, for quick comparisons")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override n of a full-length workload (a smaller case of the same "
                          "shape, e.g. for profiling)")
@@ -710,7 +723,7 @@ def main():
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    res = time_attention(w, args, dev, rank, world, True, args.steps, args.warmup)
+    res = time_attention(w, args, dev, rank, world, not args.no_e2e, args.steps, args.warmup)
     if world > 1:
         dist.barrier(device_ids=[local_rank])
         dist.destroy_process_group()
@@ -724,7 +737,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": body["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic", "config": body["config"], "roofline": body["roofline"],
-        "step_roofline": body["step_roofline"], "calls": body["calls"], "e2e": res["e2e"],
+        "step_roofline": body["step_roofline"], "calls": body["calls"], "e2e": res.get("e2e"),
         "gpu_launches": body["gpu_launches"], "clocks": body["clocks"],
     }
     if world == 1 and not args.no_sub:

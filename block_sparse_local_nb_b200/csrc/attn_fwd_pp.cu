@@ -87,9 +87,6 @@ constexpr int kRegsCtl = 56, kRegsSoft = 224;
 constexpr int kRegsLaunch = 168;  // 65536 / 384 rounded down to a multiple of 8
 static_assert(128 * kRegsCtl + 256 * kRegsSoft <= kThreads * kRegsLaunch, "register budget");
 
-// Coefficients of 2^f ~ 1 + f (c1 + f (c2 + f c3)) on [-1/2, 1/2].
-constexpr float kC1 = 0.6932829022407532f, kC2 = 0.2422109693288803f, kC3 = 0.055009059607982635f;
-
 struct Params {
   AttnArgs a;
   int nitems2;  // work items (256-row pairs of tiles) per (batch, head)
@@ -227,22 +224,6 @@ __device__ int issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t
     if (used) ++qt;
   }
   return 0;
-}
-
-// 2^x on the FMA pipe for a pair (see the file comment); x <= 64 after the clamp.
-__device__ __forceinline__ float2 exp2_fma(float2 x) {
-  x.x = fminf(fmaxf(x.x, -127.f), 64.f);
-  x.y = fminf(fmaxf(x.y, -127.f), 64.f);
-  const float2 M = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23: adding it rounds to an integer
-  const float2 t = __fadd2_rn(x, M);
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
-  float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
-  q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
-  // the low bits of t hold n: shifting them into the exponent field scales q by 2^n
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 // Softmax and epilogue warpgroup of slot s: thread = tile row r (TMEM lane r).

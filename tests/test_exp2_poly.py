@@ -1,4 +1,4 @@
-"""The forward kernel's 2^x on the FMA pipe (d = 64 kernel, attn_fwd_pp.cu):
+"""The attention kernels' 2^x on the FMA pipe (exp2_fma in sm100.cuh):
 Cody-Waite range reduction x = n + f with n = round(x), 2^f on [-1/2, 1/2] by
 a degree-3 polynomial with constant term 1, the exponent added as an integer.
 The coefficients are read from the CUDA source and the same float32 steps are
@@ -14,17 +14,17 @@ import pytest
 
 from tests.conftest import ROOT
 
-SRC = os.path.join(ROOT, "block_sparse_local_nb_b200", "csrc", "attn_fwd_pp.cu")
+SRC = os.path.join(ROOT, "block_sparse_local_nb_b200", "csrc", "sm100.cuh")
 
 
 def _coefficients():
     text = open(SRC).read()
     got = {}
-    for name in ("kC1", "kC2", "kC3"):
+    for name in ("kExp2C1", "kExp2C2", "kExp2C3"):
         m = re.search(name + r"\s*=\s*([0-9.eE+-]+)f", text)
         assert m, name
         got[name] = np.float32(float(m.group(1)))
-    return got["kC1"], got["kC2"], got["kC3"]
+    return got["kExp2C1"], got["kExp2C2"], got["kExp2C3"]
 
 
 def _exp2_fma(x):

@@ -234,7 +234,7 @@ nb_status nb_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8
   nb_status st = check_device();
   if (st != NB_OK) return st;
   cudaError_t e =
-      nb::launch_tokenize_kmer(seq, len, ids, packed, k, error_word(), static_cast<cudaStream_t>(stream));
+      nb::launch_tokenize_kmer(seq, len, ids, packed, k, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
 }
 

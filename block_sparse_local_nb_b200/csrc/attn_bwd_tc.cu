@@ -47,7 +47,7 @@ constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
 // Of every four pairs of exponentials a gradient thread computes, the first
 // kEmuBwd run on the FMA pipe (exp2_fma) instead of the special-function unit.
-constexpr int kEmuBwd = 1;
+constexpr int kEmuBwd = 0;
 
 template <int D>
 struct Cfg {
@@ -66,16 +66,17 @@ struct Cfg {
   static constexpr int oQ = NKV * 2 * kTile;     // stage s: Q at oQ + 2 s kTile, dO after it
   static constexpr int oP = oQ + NS * 2 * kTile;  // P^T tile (shared-memory variant only)
   static constexpr int oDS = oP + (kPTmem ? 0 : kPT);
+  static constexpr int oStg = oDS + kPT;  // dQ staging box (one 128 x 32 fp32 box)
   // The dK/dV epilogue of an item is deferred past the next item's first
   // chunk when the next item's K/V tile has a buffer of its own (D = 64).
   static constexpr bool kDefer = NKV > 1;
-  static constexpr int oLD = oDS + kPT;  // stage s: -lse log2e, D
+  static constexpr int oLD = oStg + kSlab;  // stage s: -lse log2e, D
   static constexpr int oBar = oLD + NS * 1024;
   static constexpr int bKVFull = 0, bKVFree = bKVFull + NKV, bQDFull = bKVFree + NKV,
                        bQDFree = bQDFull + NS, bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1,
                        bPDSFull = bSDPFree + 1, bPDSFree = bPDSFull + 1, bDQFull = bPDSFree + 1,
                        bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
-                       bOutFull = bDKVFree + 1,
+                       bStg = bDKVFree + 1, bStgFree = bStg + 1, bOutFull = bStgFree + 1,
                        bDone = bOutFull + NKV,
                        nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
@@ -88,9 +89,9 @@ struct Cfg {
   static constexpr uint32_t tP = 448;                 // P^T, bf16 pairs (TMEM-P variant)
   // registers per thread after reallocation: TMA/MMA warpgroup, each gradient
   // warpgroup, dQ warpgroup (the 16 warps share the 64K-register file)
-  static constexpr int kRegsCtl = D == 64 ? 56 : 48;
-  static constexpr int kRegsGrad = D == 64 ? 184 : 168;
-  static constexpr int kRegsDq = D == 64 ? 88 : 128;
+  static constexpr int kRegsCtl = D == 64 ? 64 : 48;
+  static constexpr int kRegsGrad = D == 64 ? 176 : 168;
+  static constexpr int kRegsDq = D == 64 ? 96 : 128;
   static_assert(128 * (kRegsCtl + 2 * kRegsGrad + kRegsDq) <= 65536, "register budget");
 };
 
@@ -102,7 +103,7 @@ struct Params {
 };
 
 struct Item {
-  int b, h, tile, L, I0, I1, nch;  // query blocks I0 .. I1 see the tile (chunks of 4 from I0)
+  int b, h, tile, L, I0, nch;
 };
 
 __device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int tile) {
@@ -115,13 +116,12 @@ __device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int ti
   x.L = min(max(L, 0), a.n);
   const int nb = a.n / kBlock;
   x.I0 = 0;
-  x.I1 = -1;
   x.nch = 0;
   if (x.tile * kRows < x.L) {
     const int kb_last = min(x.tile * 4 + 3, nb - 1);
     x.I0 = a.causal ? x.tile * 4 : max(0, x.tile * 4 - a.R);  // causal: queries at or after the keys
-    x.I1 = min(min(kb_last + a.R, nb - 1), (x.L - 1) / kBlock);
-    x.nch = (x.I1 - x.I0 + 4) / 4;
+    const int I1 = min(min(kb_last + a.R, nb - 1), (x.L - 1) / kBlock);
+    x.nch = (I1 - x.I0 + 4) / 4;
   }
   return x;
 }
@@ -143,7 +143,7 @@ __device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int 
 
 enum : int { kErrKVFree = 0x31, kErrQDFree, kErrKVFull, kErrQDFull, kErrSDPFree, kErrDQFree,
              kErrPDSFull, kErrDKVFree, kErrGQD, kErrSDPFull, kErrPDSFree, kErrDKVFull,
-             kErrDQFull, kErrDone, kErrOutFull, kErrDQFirst };
+             kErrDQFull, kErrDone, kErrStg, kErrStgFree, kErrOutFull };
 
 template <int D>
 __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tk,
@@ -501,61 +501,30 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
   return 0;
 }
 
-// Number of key tiles whose query range [I0, I1] holds query block ib of
-// (b, h): the contributions its dQ accumulates.
-__device__ __forceinline__ int block_contributors(const Params& p, int b, int h, int ib) {
-  const int lo = ib - 3 - p.a.R;
-  const int t0 = lo <= 0 ? 0 : (lo + 3) / 4;
-  const int t1 = min(p.ntiles - 1, (ib + p.a.R) / 4);
-  int n = 0;
-  for (int t = t0; t <= t1; ++t) {
-    const Item y = decode_bht(p, b, h, t);
-    n += (y.nch > 0 && y.I0 <= ib && ib <= y.I1) ? 1 : 0;
-  }
-  return n;
-}
-
-__device__ __forceinline__ void discard_l2(const void* line) {
-  asm volatile("discard.global.L2 [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(line)) : "memory");
-}
-
-// dQ warps: warp wq owns query block ib = I0 + 4c + wq of chunk c (thread =
-// query row), and its rows' dQ_c is read from TMEM.  The key tiles that see
-// block ib accumulate into its fp32 rows in global memory: the first to
-// arrive (per-block arrival counter) stores, the others wait until it has
-// completed and add with 16-byte vector reductions (L2 atomics); every one
-// then counts itself done, and the last converts the block to bf16 dQ
-// (times 1/sqrt(d)) and discards the accumulator's lines from L2, so they are
-// never written back.  Blocks outside the tile's range (the chunk's padding
-// blocks) are skipped.
+// dQ warps: thread = query row r of the chunk.
 template <int D>
-__device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem, int wq,
-                        int lane) {
+__device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
+                        uint32_t tmem, int wq, int lane, const CUtensorMap* tdq) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
+  const int r = wq * 32 + lane;
   const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-  const int nb = a.n / kBlock;
+  const bool leader = threadIdx.x == 12 * 32;
   auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
   int g = 0;
   for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
     const Item x = sched_item(p, sch, it);
     if (x.nch == 0) continue;
-    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
+    const int bh = x.b * a.heads + x.h;
     for (int c = 0; c < x.nch; ++c) {
       const int G = g + c;
-      const int ib = x.I0 + 4 * c + wq;
-      const bool contrib = ib <= x.I1;  // warp-uniform
-      const int64_t blk = bh * nb + ib;
-      float* acc = p.ws.dqacc + (blk * kBlock + lane) * D;
+      const int q0 = (x.I0 + 4 * c) * kBlock;
       if (!all_ok(mbar_wait(bar + 8 * C::bDQFull, G & 1))) return kErrDQFull;
       tc_fence_after();
-      int first = 0;
-      if (contrib) {
-        int old = 0;
-        if (lane == 0) old = atomicAdd(p.ws.arrive + blk, 1);
-        first = __shfl_sync(0xffffffffu, old, 0) == 0;
-      }
+      // dQ_c through the staging box, one 32-column box per pass; the row is read
+      // from TMEM 64 columns at a time and its TMEM released after the last read
+      uint8_t* stg = gbase + C::oStg;
 #pragma unroll
       for (int grp = 0; grp < D / 64; ++grp) {
         float v[2][32];
@@ -568,61 +537,25 @@ __device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint32
           tc_fence_before();
           mbar_arrive(bar + 8 * C::bDQFree);
         }
-        if (!contrib) continue;
-        if (first) {
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj)
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * grp + jj;      // box (32 columns) within the row
+          const int k = G * (D / 32) + j;  // global pass index
+          if (!all_ok(mbar_wait(bar + 8 * C::bStgFree, (k & 1) ^ 1))) return kErrStgFree;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              *reinterpret_cast<float4*>(acc + 64 * grp + 32 * jj + 4 * u) =
-                  make_float4(v[jj][4 * u], v[jj][4 * u + 1], v[jj][4 * u + 2], v[jj][4 * u + 3]);
-        } else {
-          if (grp == 0) {  // the first contributor's stores have completed
-            bool ok = true;
-            if (lane == 0) {
-              const uint64_t t0 = globaltimer_ns();
-              while (ld_acquire(p.ws.done + blk) < 1) {
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                  ok = false;
-                  break;
-                }
-              }
-            }
-            if (!all_ok(__shfl_sync(0xffffffffu, ok, 0))) return kErrDQFirst;
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4*>(stg + r * 128 + ((u ^ (r & 7)) << 4)) =
+                make_float4(v[jj][4 * u], v[jj][4 * u + 1], v[jj][4 * u + 2], v[jj][4 * u + 3]);
+          fence_proxy_async_smem();
+          mbar_arrive(bar + 8 * C::bStg);  // this thread's row of the box is written
+          if (leader) {
+            if (!mbar_wait(bar + 8 * C::bStg, k & 1)) return kErrStg;
+            tma_reduce_add_3d(tdq, base + C::oStg, 32 * j, q0, bh);
+            bulk_commit();
+            bulk_wait_read0();
+            mbar_arrive(bar + 8 * C::bStgFree);
           }
-#pragma unroll
-          for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              red_add_v4(acc + 64 * grp + 32 * jj + 4 * u, v[jj][4 * u], v[jj][4 * u + 1],
-                         v[jj][4 * u + 2], v[jj][4 * u + 3]);
         }
-      }
-      if (!contrib) continue;
-      __threadfence();  // this thread's stores / additions before the completion count
-      __syncwarp();
-      int prev = 0, need = 0;
-      if (lane == 0) {
-        prev = atomicAdd(p.ws.done + blk, 1);
-        need = block_contributors(p, x.b, x.h, ib);
-      }
-      prev = __shfl_sync(0xffffffffu, prev, 0);
-      need = __shfl_sync(0xffffffffu, need, 0);
-      if (prev == need - 1) {  // the last contribution: dQ = bf16(accumulator / sqrt(d))
-        __threadfence();
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.dq) + (blk * kBlock + lane) * D;
-#pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch) {
-          const float4 y0 = __ldcg(reinterpret_cast<const float4*>(acc + 8 * ch));
-          const float4 y1 = __ldcg(reinterpret_cast<const float4*>(acc + 8 * ch + 4));
-          *reinterpret_cast<uint4*>(out + 8 * ch) =
-              make_uint4(pack_bf16(y0.x * a.scale, y0.y * a.scale),
-                         pack_bf16(y0.z * a.scale, y0.w * a.scale),
-                         pack_bf16(y1.x * a.scale, y1.y * a.scale),
-                         pack_bf16(y1.z * a.scale, y1.w * a.scale));
-        }
-#pragma unroll
-        for (int l = 0; l < D * 4 / 128; ++l) discard_l2(acc + 32 * l);
       }
     }
     g += x.nch;
@@ -634,7 +567,7 @@ template <int D, bool kCausal>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                        const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
-                       const __grid_constant__ CUtensorMap tdk,
+                       const __grid_constant__ CUtensorMap tdq, const __grid_constant__ CUtensorMap tdk,
                        const __grid_constant__ CUtensorMap tdv, const Params p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -661,6 +594,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDQFree, 128);
     mbar_init(bar + 8 * C::bDKVFull, 1);
     mbar_init(bar + 8 * C::bDKVFree, 256);
+    mbar_init(bar + 8 * C::bStg, 128);
+    mbar_init(bar + 8 * C::bStgFree, 1);
     for (int i = 0; i < C::NKV; ++i) mbar_init(bar + 8 * (C::bOutFull + i), 256);
     mbar_init(bar + 8 * C::bDone, 2);  // one commit per MMA-issuing thread
     fence_barrier_init();
@@ -671,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tv);
       prefetch_tmap(&tq);
       prefetch_tmap(&tdo);
+      prefetch_tmap(&tdq);
       prefetch_tmap(&tdk);
       prefetch_tmap(&tdv);
     }
@@ -718,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   } else {
     regs_dec<C::kRegsDq>();
-    const int err = dq_warps<D>(p, sch, base, tmem, warp & 3, lane);
+    const int err = dq_warps<D>(p, sch, base, gbase, tmem, warp & 3, lane, &tdq);
     if (err) record_error(p.a.err, err);
     pdl_trigger();  // this CTA's work is issued: the next kernel may start launching
     __syncthreads();
@@ -731,12 +667,13 @@ cudaError_t launch(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
   const int64_t heads_total = static_cast<int64_t>(a.batch) * a.heads;
   Params p;
   p.a = a;
-  p.ws = bwd_workspace(a.workspace, rows, D);
-  CUtensorMap tk, tv, tq, tdo, tdk, tdv;
+  p.ws = bwd_workspace(a.workspace, rows);
+  CUtensorMap tk, tv, tq, tdo, tdq, tdk, tdv;
   if (!make_tmap_bf16_rows(&tk, a.k, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tv, a.v, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tq, a.q, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tdo, a.dout, D, a.n, heads_total, kRows) ||
+      !make_tmap_rows(&tdq, p.ws.dqacc, true, D, a.n, heads_total, 32, kRows) ||
       !make_tmap_bf16_rows(&tdk, a.dk, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tdv, a.dv, D, a.n, heads_total, kRows))
     return cudaErrorInvalidValue;
@@ -750,7 +687,7 @@ cudaError_t launch(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(items < num_sms() ? items : num_sms());
   return launch_pdl(kernel, dim3(grid), dim3(kThreads), C::kSmem, stream, tk, tv, tq,
-                    tdo, tdk, tdv, p);
+                    tdo, tdq, tdk, tdv, p);
 }
 
 }  // namespace

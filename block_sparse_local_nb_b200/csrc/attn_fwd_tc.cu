@@ -586,7 +586,7 @@ cudaError_t launch(const AttnArgs& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t stream) {
-  return a.d == 64 ? launch_attn_fwd_pp(a, stream) : launch<128>(a, stream);
+  return a.d == 64 ? launch<64>(a, stream) : launch<128>(a, stream);
 }
 
 }  // namespace nb

@@ -43,29 +43,19 @@ bool make_tmap_rows(CUtensorMap* m, const void* base, bool f32, int d, int64_t n
                     int64_t heads_total, int box_cols, int box_rows);
 int num_sms();  // SM count of the current device (cached)
 
-// Backward workspace (each region 256-byte aligned):
-//   [-D: rows fp32][-lse*log2(e): rows fp32][dQ accumulator: rows*d fp32]
-//   [per 32-row query block: arrivals int32, completions int32].
-// The counters let the key tiles that add into one query block elect the
-// first (which stores instead of adding, so the accumulator needs no
-// clearing) and the last (which converts the block's dQ to bf16).
+// Backward workspace: [-D: rows fp32][-lse*log2(e): rows fp32][dQ accumulator: rows*d fp32],
+// each region 256-byte aligned.
 struct BwdWorkspace {
   float* D;      // negated row term -D_i
   float* nlse2;
   float* dqacc;
-  int* arrive;   // [rows / 32]
-  int* done;     // [rows / 32]
 };
-__host__ __device__ inline BwdWorkspace bwd_workspace(void* ws, int64_t rows, int d) {
+__host__ __device__ inline BwdWorkspace bwd_workspace(void* ws, int64_t rows) {
   BwdWorkspace w;
   uint8_t* p = static_cast<uint8_t*>(ws);
-  const int64_t r4 = align_up(rows * 4, 256);
   w.D = reinterpret_cast<float*>(p);
-  w.nlse2 = reinterpret_cast<float*>(p + r4);
-  w.dqacc = reinterpret_cast<float*>(p + 2 * r4);
-  const int64_t c0 = 2 * r4 + align_up(rows * d * 4, 256);
-  w.arrive = reinterpret_cast<int*>(p + c0);
-  w.done = reinterpret_cast<int*>(p + c0 + align_up(rows / 32 * 4, 256));
+  w.nlse2 = reinterpret_cast<float*>(p + align_up(rows * 4, 256));
+  w.dqacc = reinterpret_cast<float*>(p + 2 * align_up(rows * 4, 256));
   return w;
 }
 cudaError_t launch_bwd_main_tc(const AttnArgs& a, int64_t rows, cudaStream_t stream);
@@ -105,7 +95,7 @@ nb_status bwd_pointer_checks(const void* q, const void* k, const void* v, const 
 nb_status device_check();  // the current device is an sm_100 GPU
 
 cudaError_t launch_tokenize_kmer(const uint8_t* seq, int64_t len, uint16_t* ids, uint8_t* packed,
-                                 int k, int* err, cudaStream_t stream);
+                                 int k, cudaStream_t stream);
 cudaError_t launch_tokenize_batch(const uint8_t* seqs, const int64_t* offsets, int batch, int k,
                                   int64_t* ids, int32_t* lengths, int n_pad, cudaStream_t stream);
 cudaError_t launch_attn_fwd_f32(const AttnArgs& a, cudaStream_t stream);

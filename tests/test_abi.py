@@ -94,10 +94,9 @@ def test_fwd_empty_problem_is_a_no_op(lib):
 def test_bwd_workspace_size(lib):
     ws = lib.nb_attn_bwd_workspace_size(4, 12, 4096, 64, BF16)
     rows = 4 * 12 * 4096
-    # row term D, -lse*log2(e), the fp32 dQ accumulator and two int32 counters
-    # per 32-row query block, each region 256-byte aligned
-    need = 2 * rows * 4 + rows * 64 * 4 + 2 * (rows // 32) * 4
-    assert need <= ws < need + 5 * 256
+    # row term D, -lse*log2(e) and the fp32 dQ accumulator, each 256-byte aligned
+    assert ws >= 2 * rows * 4 + rows * 64 * 4
+    assert ws < 2 * rows * 4 + rows * 64 * 4 + 3 * 256
     assert lib.nb_attn_bwd_workspace_size(1, 1, 33, 64, BF16) == 0  # invalid n
     assert lib.nb_attn_bwd_workspace_size(0, 1, 64, 64, BF16) == 0
 

@@ -20,6 +20,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// The same rounding (to nearest, ties to even; finite inputs) with integer
+// operations only, for code whose bf16 conversions would otherwise queue on
+// the pipe that also computes 2^x.
+__device__ __forceinline__ uint32_t pack_bf16_int(float lo, float hi) {
+  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+  a += 0x7FFFu + ((a >> 16) & 1u);
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  return __byte_perm(a, b, 0x7632);  // the high halves: a's in bits 15..0, b's in 31..16
+}
+
 namespace sm100 {
 
 // ------------------------------------------------------------------ timing

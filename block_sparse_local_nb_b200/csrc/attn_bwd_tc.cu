@@ -45,11 +45,6 @@ constexpr int kThreads = 512;
 constexpr int kRows = 128;        // keys per item, queries per chunk
 constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
-// Of every four pairs of exponentials a gradient thread computes, the first
-// kEmuBwd run on the FMA pipe (exp2_fma) instead of the special-function unit.
-constexpr int kEmuBwd = 0;
-// P and dS rounded to bf16 with integer operations instead of conversions.
-constexpr bool kIntPackBwd = false;
 
 template <int D>
 struct Cfg {
@@ -437,12 +432,11 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
                                     sl, nv[e]);  // -inf for padding queries -> P = 0
               if (8 * cc + 2 * e < cut) x.x = -INFINITY;
               if (8 * cc + 2 * e + 1 < cut) x.y = -INFINITY;
-              const float2 pe =
-                  e < kEmuBwd ? exp2_fma(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
               const float2 de = __fmul2_rn(
                   pe, __fadd2_rn(make_float2(dp[8 * cc + 2 * e], dp[8 * cc + 2 * e + 1]), nd[e]));
-              wp[16 * jj + 4 * cc + e] = kIntPackBwd ? pack_bf16_int(pe.x, pe.y) : pack_bf16(pe.x, pe.y);
-              ws[16 * jj + 4 * cc + e] = kIntPackBwd ? pack_bf16_int(de.x, de.y) : pack_bf16(de.x, de.y);
+              wp[16 * jj + 4 * cc + e] = pack_bf16(pe.x, pe.y);
+              ws[16 * jj + 4 * cc + e] = pack_bf16(de.x, de.y);
             }
           } else {
 #pragma unroll

@@ -58,11 +58,6 @@ constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 64 bf16
 constexpr float kTau = 8.0f;      // lazy-rescale threshold, log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-// Of every eight pairs of exponentials a softmax thread computes, the first
-// kEmuFwd run on the FMA pipe (exp2_fma) instead of the special-function unit.
-constexpr int kEmuFwd = 0;
-// P rounded to bf16 with integer operations instead of conversions.
-constexpr bool kIntPackFwd = false;
 
 template <int D>
 struct Cfg {
@@ -421,10 +416,9 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
 #pragma unroll
           for (int i = 0; i < 16; ++i) {  // pairs of keys, packed fp32x2 arithmetic
             const float2 xv = __ffma2_rn(make_float2(s[j][2 * i], s[j][2 * i + 1]), sl, nm);
-            const float2 pv = (i & 7) < kEmuFwd ? exp2_fma(xv)
-                                                : make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
+            const float2 pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
             ls[i & 1] = __fadd2_rn(ls[i & 1], pv);
-            w[16 * j + i] = kIntPackFwd ? pack_bf16_int(pv.x, pv.y) : pack_bf16(pv.x, pv.y);
+            w[16 * j + i] = pack_bf16(pv.x, pv.y);
           }
         } else {
 #pragma unroll

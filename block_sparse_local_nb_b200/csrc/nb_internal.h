@@ -100,7 +100,6 @@ cudaError_t launch_tokenize_batch(const uint8_t* seqs, const int64_t* offsets, i
                                   int64_t* ids, int32_t* lengths, int n_pad, cudaStream_t stream);
 cudaError_t launch_attn_fwd_f32(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t stream);
-cudaError_t launch_attn_fwd_pp(const AttnArgs& a, cudaStream_t stream);  // d = 64
 cudaError_t launch_attn_bwd_bf16(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace nb

@@ -20,16 +20,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// The same rounding (to nearest, ties to even; finite inputs) with integer
-// operations only, for code whose bf16 conversions would otherwise queue on
-// the pipe that also computes 2^x.
-__device__ __forceinline__ uint32_t pack_bf16_int(float lo, float hi) {
-  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-  a += 0x7FFFu + ((a >> 16) & 1u);
-  b += 0x7FFFu + ((b >> 16) & 1u);
-  return __byte_perm(a, b, 0x7632);  // the high halves: a's in bits 15..0, b's in 31..16
-}
-
 namespace sm100 {
 
 // ------------------------------------------------------------------ timing
@@ -78,13 +68,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-// Load with acquire semantics at GPU scope (pairs with a release by another CTA).
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // Record the first error code seen by any thread (0 = none).
 __device__ __forceinline__ void record_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
@@ -112,13 +95,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
           dst),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
       : "memory");
-}
-// Four consecutive floats added into global memory (an L2 atomic, relaxed;
-// the address is 16-byte aligned).
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
 }
 // 3-D tiled reduce-add of an fp32 shared-memory tile into global memory.
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, uint32_t src, int x, int y,
@@ -286,30 +262,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x for a pair on the FMA pipe instead of the special-function unit
-// (exponentials are shared between the two pipes when the latter is the
-// bottleneck).  Cody and Waite's range reduction: x = n + f with n = round(x)
-// (adding 1.5 * 2^23 rounds to an integer and leaves n in the low bits), 2^f
-// on [-1/2, 1/2] by a degree-3 polynomial with constant term 1 whose other
-// coefficients minimise the maximum relative error (1.0e-4), solved as a
-// linear program over a fine grid of f; 2^n is added to the exponent field as
-// an integer.  x is clamped to [-127, 64]: -inf (a masked key) gives exactly 0
-// (n = -127, f = 0, 1.0 shifted down to +0), +64 is the largest result.
-constexpr float kExp2C1 = 0.6932829022407532f, kExp2C2 = 0.2422109693288803f,
-                kExp2C3 = 0.055009059607982635f;
-__device__ __forceinline__ float2 exp2_fma(float2 x) {
-  x.x = fminf(fmaxf(x.x, -127.f), 64.f);
-  x.y = fminf(fmaxf(x.y, -127.f), 64.f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
-  float2 q = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-  q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
-  q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 // ------------------------------------------------------------- descriptors

@@ -56,27 +56,24 @@ struct Cfg {
   // free as soon as its gradient products complete.
   static constexpr bool kPTmem = D == 64;
   static constexpr int NKV = D == 64 ? 2 : 1;  // K/V tile buffers
-  // dQ staging boxes: with two, a box is written while the previous one's
-  // reduce-add is still reading shared memory (D = 64 then keeps two Q/dO stages)
-  static constexpr int kNStg = D == 64 ? 1 : 1;
-  static constexpr int NS = D == 64 ? (kNStg == 2 ? 2 : 3) : 1;  // Q/dO chunk stages
+  static constexpr int NS = D == 64 ? 3 : 1;   // Q/dO chunk stages
   static constexpr int kTile = kRows * D * 2;  // one [128 x D] bf16 tile
   static constexpr int kPT = kRows * kRows * 2;  // one [128 x 128] bf16 tile
   static constexpr int oK = 0;                   // buffer i: K at oK + 2 i kTile, V after it
   static constexpr int oQ = NKV * 2 * kTile;     // stage s: Q at oQ + 2 s kTile, dO after it
   static constexpr int oP = oQ + NS * 2 * kTile;  // P^T tile (shared-memory variant only)
   static constexpr int oDS = oP + (kPTmem ? 0 : kPT);
-  static constexpr int oStg = oDS + kPT;  // dQ staging boxes (128 x 32 fp32 each)
+  static constexpr int oStg = oDS + kPT;  // dQ staging box (one 128 x 32 fp32 box)
   // The dK/dV epilogue of an item is deferred past the next item's first
   // chunk when the next item's K/V tile has a buffer of its own (D = 64).
   static constexpr bool kDefer = NKV > 1;
-  static constexpr int oLD = oStg + kNStg * kSlab;  // stage s: -lse log2e, D
+  static constexpr int oLD = oStg + kSlab;  // stage s: -lse log2e, D
   static constexpr int oBar = oLD + NS * 1024;
   static constexpr int bKVFull = 0, bKVFree = bKVFull + NKV, bQDFull = bKVFree + NKV,
                        bQDFree = bQDFull + NS, bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1,
                        bPDSFull = bSDPFree + 1, bPDSFree = bPDSFull + 1, bDQFull = bPDSFree + 1,
                        bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
-                       bStg = bDKVFree + 1, bStgFree = bStg + kNStg, bOutFull = bStgFree + kNStg,
+                       bStg = bDKVFree + 1, bStgFree = bStg + 1, bOutFull = bStgFree + 1,
                        bDone = bOutFull + NKV,
                        nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
@@ -540,26 +537,19 @@ __device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint8_
         for (int jj = 0; jj < 2; ++jj) {
           const int j = 2 * grp + jj;      // box (32 columns) within the row
           const int k = G * (D / 32) + j;  // global pass index
-          const int sb = k % C::kNStg, ph = (k / C::kNStg) & 1;  // staging box and its phase
-          if (!all_ok(mbar_wait(bar + 8 * (C::bStgFree + sb), ph ^ 1))) return kErrStgFree;
-          uint8_t* box = stg + sb * kSlab;
+          if (!all_ok(mbar_wait(bar + 8 * C::bStgFree, (k & 1) ^ 1))) return kErrStgFree;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<float4*>(box + r * 128 + ((u ^ (r & 7)) << 4)) =
+            *reinterpret_cast<float4*>(stg + r * 128 + ((u ^ (r & 7)) << 4)) =
                 make_float4(v[jj][4 * u], v[jj][4 * u + 1], v[jj][4 * u + 2], v[jj][4 * u + 3]);
           fence_proxy_async_smem();
-          mbar_arrive(bar + 8 * (C::bStg + sb));  // this thread's row of the box is written
+          mbar_arrive(bar + 8 * C::bStg);  // this thread's row of the box is written
           if (leader) {
-            if (!mbar_wait(bar + 8 * (C::bStg + sb), ph)) return kErrStg;
-            tma_reduce_add_3d(tdq, base + C::oStg + sb * kSlab, 32 * j, q0, bh);
+            if (!mbar_wait(bar + 8 * C::bStg, k & 1)) return kErrStg;
+            tma_reduce_add_3d(tdq, base + C::oStg, 32 * j, q0, bh);
             bulk_commit();
-            if (C::kNStg == 1) {
-              bulk_wait_read0();
-              mbar_arrive(bar + 8 * C::bStgFree);
-            } else if (k > 0) {  // the previous box's reduce has read it: release that box
-              bulk_wait_read1();
-              mbar_arrive(bar + 8 * (C::bStgFree + (k - 1) % C::kNStg));
-            }
+            bulk_wait_read0();
+            mbar_arrive(bar + 8 * C::bStgFree);
           }
         }
       }
@@ -601,10 +591,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDQFree, 128);
     mbar_init(bar + 8 * C::bDKVFull, 1);
     mbar_init(bar + 8 * C::bDKVFree, 256);
-    for (int i = 0; i < C::kNStg; ++i) {
-      mbar_init(bar + 8 * (C::bStg + i), 128);
-      mbar_init(bar + 8 * (C::bStgFree + i), 1);
-    }
+    mbar_init(bar + 8 * C::bStg, 128);
+    mbar_init(bar + 8 * C::bStgFree, 1);
     for (int i = 0; i < C::NKV; ++i) mbar_init(bar + 8 * (C::bOutFull + i), 256);
     mbar_init(bar + 8 * C::bDone, 2);  // one commit per MMA-issuing thread
     fence_barrier_init();

@@ -11,10 +11,12 @@ from .binding import (  # noqa: F401
     NB_F32,
     NbError,
     attn_bwd_workspace_size,
+    attn_fwd_bwd_host_workspace_size,
     lib,
     nb_attn_bwd,
     nb_attn_bwd_causal,
     nb_attn_fwd,
+    nb_attn_fwd_bwd_host,
     nb_attn_fwd_causal,
     nb_batch_ceiling,
     nb_kernel_error,

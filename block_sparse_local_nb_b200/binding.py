@@ -33,6 +33,8 @@ _SIGS = [
                          _I, _I, _I, _I, _I, _I, _P]),
     ("nb_attn_bwd_causal", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                 _I, _I, _I, _I, _I, _I, _P]),
+    ("nb_attn_fwd_bwd_host_workspace_size", ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    ("nb_attn_fwd_bwd_host", _I, [_P] * 11 + [ctypes.c_size_t] + [_I] * 7 + [_P]),
     ("nb_tokenize_kmer", _I, [_P, ctypes.c_int64, _P, _P, _I, _P]),
     ("nb_tokenize_batch", _I, [_P, _P, _I, _I, _P, _P, _I, _P]),
     ("nb_batch_ceiling", _I, [_P, _I, _I, ctypes.POINTER(ctypes.c_int32)]),
@@ -136,6 +138,23 @@ def nb_attn_bwd_causal(q, k, v, o, dout, lse, lengths, dq, dk, dv, workspace, wo
                                   workspace_bytes, batch, heads, n, d, R, dtype, _stream(stream))
     if check:
         _check(st, "nb_attn_bwd_causal")
+    return st
+
+
+def attn_fwd_bwd_host_workspace_size(batch, heads, n, d, dtype) -> int:
+    return int(lib().nb_attn_fwd_bwd_host_workspace_size(batch, heads, n, d, dtype))
+
+
+def nb_attn_fwd_bwd_host(q, k, v, dout, lengths, o, lse, dq, dk, dv, workspace, workspace_bytes,
+                         batch, heads, n, d, R, dtype, causal=False, stream=None, check=True):
+    """Forward + backward of HOST tensors (pinned CPU tensors or addresses); the
+    workspace is a device buffer.  Asynchronous on `stream`."""
+    st = lib().nb_attn_fwd_bwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lengths),
+                                    _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                                    _ptr(workspace), workspace_bytes, batch, heads, n, d, R,
+                                    dtype, 1 if causal else 0, _stream(stream))
+    if check:
+        _check(st, "nb_attn_fwd_bwd_host")
     return st
 
 

@@ -17,7 +17,8 @@
  *     "Architecture Size"): 2-bit bases, sliding-window 6-mer IDs.
  *
  * Conventions shared by every call:
- *   - Every pointer argument is a DEVICE pointer unless stated otherwise.  The
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise (only
+ *     nb_attn_fwd_bwd_host and nb_batch_ceiling take host tensors).  The
  *     caller owns every buffer; no call allocates device memory.  The library
  *     keeps no state between calls except per-device caches (device
  *     properties, the device addresses of its two __device__ variables) and
@@ -155,6 +156,45 @@ NB_API nb_status nb_attn_bwd_causal(const void* q, const void* k, const void* v,
                                     void* dq, void* dk, void* dv, void* workspace,
                                     size_t workspace_bytes, int batch, int heads, int n, int d,
                                     int R, int dtype, void* stream);
+
+/*
+ * nb_attn_fwd_bwd_host - forward then backward (nb_attn_fwd, nb_attn_bwd, or
+ * their causal forms when `causal` is non-zero) of tensors that live in HOST
+ * memory: the training step of one attention layer for a caller whose
+ * activations are on the host.  (NucleoByte page, section 3: the forward and
+ * "Custom Backpropagation"; the overlap of transfers with compute is this
+ * library's, the page has none.)
+ * q, k, v, dout  in : host [batch, heads, n, d] bf16.
+ * lengths        in : host int32 [batch] or NULL (see conventions).
+ * o              out: host [batch, heads, n, d] bf16.
+ * lse            out: host [batch, heads, n] fp32, or NULL when not wanted.
+ * dq, dk, dv     out: host [batch, heads, n, d] bf16.
+ * workspace          : DEVICE scratch of at least
+ *                      nb_attn_fwd_bwd_host_workspace_size(...) bytes,
+ *                      256-byte aligned, owned by the caller; contents on entry
+ *                      do not matter.  It holds a few chunks at a time, not the
+ *                      whole problem.
+ * The (batch, head) slices are cut into about eight chunks; chunk i + 1 is
+ * copied to the device while chunk i computes on `stream` and chunk i - 1 is
+ * copied back, on two streams the call creates and releases.  The host
+ * buffers must be page-locked (cudaHostAlloc / cudaHostRegister) for the
+ * copies to overlap; pageable memory gives the same results, serialised.
+ * The call is asynchronous: it returns once everything is queued, and the
+ * outputs are complete when `stream` reaches the point where the call was
+ * made (synchronise it before reading them).  The host inputs must stay
+ * unchanged and the outputs unread until then.  Results equal those of
+ * nb_attn_fwd + nb_attn_bwd on device copies of the same tensors (dQ up to
+ * the order of its fp32 atomic additions).
+ * Errors: as nb_attn_bwd (NB_BF16 only; NB_F32 returns NB_ERR_UNSUPPORTED);
+ * a CUDA failure after some chunks were queued returns NB_ERR_CUDA with the
+ * queued work still ordered before later work on `stream`.
+ */
+NB_API size_t nb_attn_fwd_bwd_host_workspace_size(int batch, int heads, int n, int d, int dtype);
+NB_API nb_status nb_attn_fwd_bwd_host(const void* q, const void* k, const void* v,
+                                      const void* dout, const int32_t* lengths, void* o,
+                                      float* lse, void* dq, void* dk, void* dv, void* workspace,
+                                      size_t workspace_bytes, int batch, int heads, int n, int d,
+                                      int R, int dtype, int causal, void* stream);
 
 /*
  * nb_attn_bwd_noalloc - nb_attn_bwd for callers that cannot allocate device

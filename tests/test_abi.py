@@ -197,3 +197,39 @@ def test_noalloc_rejects_on_the_host(lib):
     assert fn(*nulls, 0, 1, 64, 64, 1, BF16, None) == NB_OK  # empty problem
     ptrs = [16] * 6 + [None] + [16, 16, 24]  # dv not 16-byte aligned
     assert fn(*ptrs, 1, 1, 64, 64, 1, BF16, None) == NB_ERR_MISALIGNED
+
+
+def _host(lib, ws=256, ws_bytes=1 << 40, q=16, dq=16, dtype=BF16, n=64, d=64, R=1, batch=1):
+    fn = lib.nb_attn_fwd_bwd_host
+    return fn(q, 16, 16, 16, None, 16, None, dq, 16, 16, ws, ws_bytes, batch, 2, n, d, R, dtype, 0,
+              None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), NB_ERR_INVALID_ARG),
+    (dict(dq=None), NB_ERR_INVALID_ARG),
+    (dict(n=40), NB_ERR_INVALID_ARG),
+    (dict(R=-1), NB_ERR_INVALID_ARG),
+    (dict(d=96), NB_ERR_UNSUPPORTED),
+    (dict(dtype=F32), NB_ERR_UNSUPPORTED),
+    (dict(ws=None), NB_ERR_WORKSPACE),
+    (dict(ws=272), NB_ERR_WORKSPACE),
+    (dict(ws_bytes=1024), NB_ERR_WORKSPACE),
+    (dict(batch=0), NB_OK),
+])
+def test_host_step_rejects_invalid_arguments(lib, kw, status):
+    assert _host(lib, **kw) == status
+
+
+def test_host_step_workspace_holds_a_few_chunks(lib):
+    """The host entry point's device scratch holds three chunks, not the whole
+    problem: 1 x 8 x 2^20 x 64 is cut into eight one-head chunks."""
+    n, d = 1 << 20, 64
+    ws = lib.nb_attn_fwd_bwd_host_workspace_size(1, 8, n, d, BF16)
+    one_head = 8 * n * d * 2 + n * 4 + lib.nb_attn_bwd_workspace_size(1, 1, n, d, BF16)
+    assert 3 * one_head <= ws <= 3 * one_head + 64 * 1024
+    assert lib.nb_attn_fwd_bwd_host_workspace_size(1, 8, n, d, F32) == 0
+    assert lib.nb_attn_fwd_bwd_host_workspace_size(0, 8, n, d, BF16) == 0
+    # a single slice: one chunk, one slot
+    one = lib.nb_attn_fwd_bwd_host_workspace_size(1, 1, 64, d, BF16)
+    assert one < 2 * (8 * 64 * d * 2 + 64 * 4 + lib.nb_attn_bwd_workspace_size(1, 1, 64, d, BF16))

@@ -485,7 +485,7 @@ def time_attention(w, args, dev, rank, world, with_e2e, steps, warmup):
         for name in ("q", "k", "v", "do", "o", "lse", "dq", "dk", "dv", "ws"):
             st.pop(name)
         torch.cuda.empty_cache()
-        hws_bytes = nb.attn_fwd_bwd_host_workspace_size(B, H, N, D, dt_code)
+        hws_bytes = nb.attn_fwd_bwd_host_workspace_size(B, H, N, D, R, dt_code)
         hws = torch.empty(hws_bytes, dtype=torch.uint8, device=dev)
     e_steps = max(1, min(steps, 5))
     e_start = torch.cuda.Event(enable_timing=True)

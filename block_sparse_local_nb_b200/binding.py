@@ -33,7 +33,7 @@ _SIGS = [
                          _I, _I, _I, _I, _I, _I, _P]),
     ("nb_attn_bwd_causal", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                 _I, _I, _I, _I, _I, _I, _P]),
-    ("nb_attn_fwd_bwd_host_workspace_size", ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    ("nb_attn_fwd_bwd_host_workspace_size", ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     ("nb_attn_fwd_bwd_host", _I, [_P] * 11 + [ctypes.c_size_t] + [_I] * 7 + [_P]),
     ("nb_tokenize_kmer", _I, [_P, ctypes.c_int64, _P, _P, _I, _P]),
     ("nb_tokenize_batch", _I, [_P, _P, _I, _I, _P, _P, _I, _P]),
@@ -141,8 +141,8 @@ def nb_attn_bwd_causal(q, k, v, o, dout, lse, lengths, dq, dk, dv, workspace, wo
     return st
 
 
-def attn_fwd_bwd_host_workspace_size(batch, heads, n, d, dtype) -> int:
-    return int(lib().nb_attn_fwd_bwd_host_workspace_size(batch, heads, n, d, dtype))
+def attn_fwd_bwd_host_workspace_size(batch, heads, n, d, R, dtype) -> int:
+    return int(lib().nb_attn_fwd_bwd_host_workspace_size(batch, heads, n, d, R, dtype))
 
 
 def nb_attn_fwd_bwd_host(q, k, v, dout, lengths, o, lse, dq, dk, dv, workspace, workspace_bytes,

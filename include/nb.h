@@ -174,22 +174,29 @@ NB_API nb_status nb_attn_bwd_causal(const void* q, const void* k, const void* v,
  *                      256-byte aligned, owned by the caller; contents on entry
  *                      do not matter.  It holds a few chunks at a time, not the
  *                      whole problem.
- * The (batch, head) slices are cut into about eight chunks; chunk i + 1 is
+ * The work is cut into about 32 chunks: groups of whole (batch, head) slices,
+ * or, when there are fewer than 32 slices, windows of one slice's sequence
+ * (the rows a window owns plus 2R blocks of context on each side, which make
+ * the owned rows' results exact; only those are copied back).  Chunk i + 1 is
  * copied to the device while chunk i computes on `stream` and chunk i - 1 is
  * copied back, on two streams the call creates and releases.  The host
  * buffers must be page-locked (cudaHostAlloc / cudaHostRegister) for the
  * copies to overlap; pageable memory gives the same results, serialised.
+ * `lengths` is also read on the host during the call (window lengths).
  * The call is asynchronous: it returns once everything is queued, and the
  * outputs are complete when `stream` reaches the point where the call was
  * made (synchronise it before reading them).  The host inputs must stay
  * unchanged and the outputs unread until then.  Results equal those of
- * nb_attn_fwd + nb_attn_bwd on device copies of the same tensors (dQ up to
- * the order of its fp32 atomic additions).
+ * nb_attn_fwd + nb_attn_bwd on device copies of the same tensors, up to the
+ * order of fp32 additions: dQ's atomic additions and, in windows, the online
+ * softmax and accumulation over the same keys from another first chunk.  The
+ * workspace size depends on R (through the windows' context).
  * Errors: as nb_attn_bwd (NB_BF16 only; NB_F32 returns NB_ERR_UNSUPPORTED);
  * a CUDA failure after some chunks were queued returns NB_ERR_CUDA with the
  * queued work still ordered before later work on `stream`.
  */
-NB_API size_t nb_attn_fwd_bwd_host_workspace_size(int batch, int heads, int n, int d, int dtype);
+NB_API size_t nb_attn_fwd_bwd_host_workspace_size(int batch, int heads, int n, int d, int R,
+                                                  int dtype);
 NB_API nb_status nb_attn_fwd_bwd_host(const void* q, const void* k, const void* v,
                                       const void* dout, const int32_t* lengths, void* o,
                                       float* lse, void* dq, void* dk, void* dv, void* workspace,

@@ -223,13 +223,16 @@ def test_host_step_rejects_invalid_arguments(lib, kw, status):
 
 def test_host_step_workspace_holds_a_few_chunks(lib):
     """The host entry point's device scratch holds three chunks, not the whole
-    problem: 1 x 8 x 2^20 x 64 is cut into eight one-head chunks."""
-    n, d = 1 << 20, 64
-    ws = lib.nb_attn_fwd_bwd_host_workspace_size(1, 8, n, d, BF16)
-    one_head = 8 * n * d * 2 + n * 4 + lib.nb_attn_bwd_workspace_size(1, 1, n, d, BF16)
-    assert 3 * one_head <= ws <= 3 * one_head + 64 * 1024
-    assert lib.nb_attn_fwd_bwd_host_workspace_size(1, 8, n, d, F32) == 0
-    assert lib.nb_attn_fwd_bwd_host_workspace_size(0, 8, n, d, BF16) == 0
-    # a single slice: one chunk, one slot
-    one = lib.nb_attn_fwd_bwd_host_workspace_size(1, 1, 64, d, BF16)
+    problem: 1 x 8 x 2^20 x 64 at R = 8 has eight slices, each cut into four
+    windows that own 8192 blocks and carry 2R = 16 blocks of context a side."""
+    n, d, R = 1 << 20, 64, 8
+    ws = lib.nb_attn_fwd_bwd_host_workspace_size(1, 8, n, d, R, BF16)
+    rows = (8192 + 4 * R) * 32  # an inner window
+    one = 8 * rows * d * 2 + rows * 4 + lib.nb_attn_bwd_workspace_size(1, 1, rows, d, BF16)
+    assert 3 * one <= ws <= 3 * one + 64 * 1024
+    assert lib.nb_attn_fwd_bwd_host_workspace_size(1, 8, n, d, R, F32) == 0
+    assert lib.nb_attn_fwd_bwd_host_workspace_size(0, 8, n, d, R, BF16) == 0
+    assert lib.nb_attn_fwd_bwd_host_workspace_size(1, 8, n, d, -1, BF16) == 0
+    # a slice too short to cut: one chunk, one slot
+    one = lib.nb_attn_fwd_bwd_host_workspace_size(1, 1, 64, d, 1, BF16)
     assert one < 2 * (8 * 64 * d * 2 + 64 * 4 + lib.nb_attn_bwd_workspace_size(1, 1, 64, d, BF16))

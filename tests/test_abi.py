@@ -199,10 +199,17 @@ def test_noalloc_rejects_on_the_host(lib):
     assert fn(*ptrs, 1, 1, 64, 64, 1, BF16, None) == NB_ERR_MISALIGNED
 
 
-def _host(lib, ws=256, ws_bytes=1 << 40, q=16, dq=16, dtype=BF16, n=64, d=64, R=1, batch=1):
+_HOST_BUF = ctypes.create_string_buffer(4096)  # real host memory for the host-side tensors
+_HB = ctypes.addressof(_HOST_BUF)
+
+
+def _host(lib, ws=None, ws_bytes=1 << 40, q=_HB, dq=_HB, dtype=BF16, n=64, d=64, R=1, batch=1):
+    """Every case is rejected before any copy or launch; the workspace (the only
+    device pointer) is NULL unless the case is about the workspace, so a change
+    in the order of the checks fails here on the host."""
     fn = lib.nb_attn_fwd_bwd_host
-    return fn(q, 16, 16, 16, None, 16, None, dq, 16, 16, ws, ws_bytes, batch, 2, n, d, R, dtype, 0,
-              None)
+    return fn(q, _HB, _HB, _HB, None, _HB, None, dq, _HB, _HB, ws, ws_bytes, batch, 2, n, d, R,
+              dtype, 0, None)
 
 
 @pytest.mark.parametrize("kw,status", [

@@ -690,7 +690,7 @@ cudaError_t launch(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_bwd_main_tc(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
-  return a.d == 64 ? launch<64>(a, rows, stream) : launch<128>(a, rows, stream);
+  return a.d == 64 ? launch<64>(a, rows, stream) : launch_bwd_main_tc_d128(a, rows, stream);
 }
 
 }  // namespace nb

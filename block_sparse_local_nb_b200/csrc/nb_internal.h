@@ -59,6 +59,8 @@ __host__ __device__ inline BwdWorkspace bwd_workspace(void* ws, int64_t rows) {
   return w;
 }
 cudaError_t launch_bwd_main_tc(const AttnArgs& a, int64_t rows, cudaStream_t stream);
+// d = 128 main kernel (64-query chunks; attn_bwd_tc_d128.cu)
+cudaError_t launch_bwd_main_tc_d128(const AttnArgs& a, int64_t rows, cudaStream_t stream);
 
 // Programmatic dependent launch.  Every kernel of this library is launched
 // with it: a kernel may begin (set up barriers, tensor memory, descriptor

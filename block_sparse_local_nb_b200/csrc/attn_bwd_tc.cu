@@ -1,5 +1,6 @@
-// Banded block-sparse local attention backward, main kernel, on the
-// 5th-generation tensor cores (tcgen05 + TMEM), bf16 in / fp32 accumulate.
+// Banded block-sparse local attention backward, main kernel for d = 64 (d = 128
+// is attn_bwd_tc_d128.cu), on the 5th-generation tensor cores (tcgen05 +
+// TMEM), bf16 in / fp32 accumulate.
 // (NucleoByte page, section 3 "Custom Backpropagation": P recomputed from the
 // stored log-sum-exp, D_i = sum_k dO_ik O_ik, dS = P (dO V^T - D); gradients of
 // shared key/value blocks accumulated with atomic adds.)
@@ -25,8 +26,8 @@
 // behind the other's barriers), warp 3 the dK/dV tile stores; warpgroups 1-2:
 // gradient warps, one warpgroup per half of the chunk's query columns, thread =
 // key row; they also stage dK (first) and dV (second) of an item in its K/V
-// buffer, for D = 64 after the next item's first chunk (so the wait for the
-// item's last products overlaps that chunk's arithmetic);
+// buffer after the next item's first chunk (so the wait for the item's last
+// products overlaps that chunk's arithmetic);
 // warpgroup 3: dQ warps, thread = query row, stage dQ_c in shared memory and
 // reduce it into global memory.  All waits are bounded (see sm100.cuh).
 #include <math.h>
@@ -48,25 +49,20 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
-  // D = 64: K/V tiles double-buffered, three Q/dO stages; P^T kept in TMEM
-  // (64 spare columns) as the A operand of dV.
-  // D = 128: TMEM is full (dQ reuses the S columns, so S/dP of chunk G + 1
-  // waits until dQ of chunk G is read out) and P^T goes through shared memory.
-  // Both stage dQ through one 128 x 32 fp32 box, so a chunk's Q/dO buffer is
-  // free as soon as its gradient products complete.
-  static constexpr bool kPTmem = D == 64;
-  static constexpr int NKV = D == 64 ? 2 : 1;  // K/V tile buffers
-  static constexpr int NS = D == 64 ? 3 : 1;   // Q/dO chunk stages
+  static_assert(D == 64, "this kernel is the d = 64 one");
+  // K/V tiles double-buffered, three Q/dO stages; P^T kept in TMEM (64 spare
+  // columns) as the A operand of dV; dQ staged through one 128 x 32 fp32 box,
+  // so a chunk's Q/dO buffer is free as soon as its gradient products complete.
+  static constexpr int NKV = 2;  // K/V tile buffers
+  static constexpr int NS = 3;   // Q/dO chunk stages
   static constexpr int kTile = kRows * D * 2;  // one [128 x D] bf16 tile
   static constexpr int kPT = kRows * kRows * 2;  // one [128 x 128] bf16 tile
   static constexpr int oK = 0;                   // buffer i: K at oK + 2 i kTile, V after it
   static constexpr int oQ = NKV * 2 * kTile;     // stage s: Q at oQ + 2 s kTile, dO after it
-  static constexpr int oP = oQ + NS * 2 * kTile;  // P^T tile (shared-memory variant only)
-  static constexpr int oDS = oP + (kPTmem ? 0 : kPT);
+  static constexpr int oDS = oQ + NS * 2 * kTile;  // dS^T tile
   static constexpr int oStg = oDS + kPT;  // dQ staging box (one 128 x 32 fp32 box)
   // The dK/dV epilogue of an item is deferred past the next item's first
-  // chunk when the next item's K/V tile has a buffer of its own (D = 64).
-  static constexpr bool kDefer = NKV > 1;
+  // chunk (the next item's K/V tile has a buffer of its own).
   static constexpr int oLD = oStg + kSlab;  // stage s: -lse log2e, D
   static constexpr int oBar = oLD + NS * 1024;
   static constexpr int bKVFull = 0, bKVFree = bKVFull + NKV, bQDFull = bKVFree + NKV,
@@ -81,14 +77,13 @@ struct Cfg {
   static constexpr int kSmem = oSched + kSchedBytes + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D;
-  static constexpr uint32_t tDQ = D == 64 ? 384 : 0;  // for D = 128, dQ reuses the S columns
-  static constexpr uint32_t tP = 448;                 // P^T, bf16 pairs (TMEM-P variant)
+  static constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D, tDQ = 384;
+  static constexpr uint32_t tP = 448;                 // P^T, bf16 pairs
   // registers per thread after reallocation: TMA/MMA warpgroup, each gradient
   // warpgroup, dQ warpgroup (the 16 warps share the 64K-register file)
-  static constexpr int kRegsCtl = D == 64 ? 64 : 48;
-  static constexpr int kRegsGrad = D == 64 ? 176 : 168;
-  static constexpr int kRegsDq = D == 64 ? 96 : 128;
+  static constexpr int kRegsCtl = 64;
+  static constexpr int kRegsGrad = 176;
+  static constexpr int kRegsDq = 96;
   static_assert(128 * (kRegsCtl + 2 * kRegsGrad + kRegsDq) <= 65536, "register budget");
 };
 
@@ -209,8 +204,6 @@ __device__ int sdp_issuer(const Params& p, const Sched& sch, uint32_t base, uint
       const uint64_t dQ = smem_desc_sw128(sQ, 0, 1024), ddO = smem_desc_sw128(sQ + C::kTile, 0, 1024);
       if (!mbar_wait(bar + 8 * (C::bQDFull + st), (G / C::NS) & 1)) return kErrQDFull;
       if (!mbar_wait(bar + 8 * C::bSDPFree, (G & 1) ^ 1)) return kErrSDPFree;
-      // D = 128: dQ of the previous chunk occupies the S columns until it is read out
-      if (D == 128 && !mbar_wait(bar + 8 * C::bDQFree, (G & 1) ^ 1)) return kErrDQFree;
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
@@ -235,7 +228,6 @@ __device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uin
   const uint32_t bar = base + C::oBar;
   constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, false, true);  // P^T dO, dS^T Q
   constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, true, true);    // dS K
-  const uint64_t dP = smem_desc_sw128(base + C::oP, 0, 1024);
   const uint64_t dSk = smem_desc_sw128(base + C::oDS, 0, 1024);      // dS^T, K-major A
   const uint64_t dSm = smem_desc_sw128(base + C::oDS, kSlab, 1024);  // dS, MN-major A
   int g = 0, tc = 0;
@@ -251,16 +243,13 @@ __device__ int grad_issuer(const Params& p, const Sched& sch, uint32_t base, uin
       const bool acc = c > 0;
       if (!mbar_wait(bar + 8 * C::bPDSFull, G & 1)) return kErrPDSFull;
       if (c == 0 && !mbar_wait(bar + 8 * C::bDKVFree, (tc & 1) ^ 1)) return kErrDKVFree;
-      if (D == 64 && !mbar_wait(bar + 8 * C::bDQFree, (G & 1) ^ 1)) return kErrDQFree;
+      if (!mbar_wait(bar + 8 * C::bDQFree, (G & 1) ^ 1)) return kErrDQFree;
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < kRows / 16; ++k) {  // k over the chunk's queries
         const uint32_t off = ((k >> 2) * kSlab + (k & 3) * 32) >> 4;
         const uint32_t mn = (k * 2048) >> 4;  // 16 rows of an MN-major operand
-        if (C::kPTmem)
-          mma_bf16_ts(tmem + C::tDV, tmem + C::tP + 8 * k, desc_add(ddO, mn), kIdKV, acc || k > 0);
-        else
-          mma_bf16_ss(tmem + C::tDV, desc_add(dP, off), desc_add(ddO, mn), kIdKV, acc || k > 0);
+        mma_bf16_ts(tmem + C::tDV, tmem + C::tP + 8 * k, desc_add(ddO, mn), kIdKV, acc || k > 0);
         mma_bf16_ss(tmem + C::tDK, desc_add(dSk, off), desc_add(dQ, mn), kIdKV, acc || k > 0);
       }
       // Q and dO are last read by the products above: their buffer can refill
@@ -444,29 +433,23 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
       // the previous chunk's dV/dK/dQ products must be done reading the P/dS tiles
       if (!all_ok(mbar_wait(bar + 8 * C::bPDSFree, (G & 1) ^ 1))) return kErrPDSFree;
 
-      uint8_t* prow = gbase + C::oP + hf * kSlab + r * 128;
       uint8_t* srow = gbase + C::oDS + hf * kSlab + r * 128;
-      if (C::kPTmem) {  // this thread's 64 queries = 32 packed columns of P^T in TMEM
-        tmem_st32u(trow + C::tP + 32 * hf, wp);
-      }
+      // this thread's 64 queries = 32 packed columns of P^T in TMEM
+      tmem_st32u(trow + C::tP + 32 * hf, wp);
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           const int ch = ((4 * jj + cc) ^ (r & 7)) << 4;
-          if (!C::kPTmem)
-            *reinterpret_cast<uint4*>(prow + ch) =
-                make_uint4(wp[16 * jj + 4 * cc], wp[16 * jj + 4 * cc + 1],
-                           wp[16 * jj + 4 * cc + 2], wp[16 * jj + 4 * cc + 3]);
           *reinterpret_cast<uint4*>(srow + ch) =
               make_uint4(ws[16 * jj + 4 * cc], ws[16 * jj + 4 * cc + 1], ws[16 * jj + 4 * cc + 2],
                          ws[16 * jj + 4 * cc + 3]);
         }
-      if (C::kPTmem) tmem_wait_st();
+      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar + 8 * C::bPDSFull);
-      if (C::kDefer && c == 0 && pend.valid) {
+      if (c == 0 && pend.valid) {
         // the previous item's epilogue: its last products completed before the
         // P/dS tiles were free, so only the TMEM read delays this chunk's products
         if ((e = epi_load(pend.tc, pend.row_valid))) return e;
@@ -474,16 +457,11 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
         pend.valid = false;
       }
     }
-    if (C::kDefer) {
-      pend = {true, tc, row_valid};
-    } else {
-      if ((e = epi_load(tc, row_valid))) return e;
-      epi_stage(tc % C::NKV);
-    }
+    pend = {true, tc, row_valid};
     g += x.nch;
     ++tc;
   }
-  if (C::kDefer && pend.valid) {
+  if (pend.valid) {
     if ((e = epi_load(pend.tc, pend.row_valid))) return e;
     epi_stage(pend.tc % C::NKV);
   }

@@ -520,7 +520,10 @@ def time_attention(w, args, dev, rank, world, with_e2e, steps, warmup):
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
     check_kernel_error(nb)
     res["e2e"] = {"value": job_throughput(alg["tokens"], e_steps, world, e2e_ms), "unit": "tokens/s",
-                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps}
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+                  "path": ("nb_attn_fwd_bwd_host on pinned host tensors (chunked copy-in / compute / "
+                           "copy-out overlap) + nb_tokenize_kmer with plain copies" if w.backward else
+                           "plain copies around nb_tokenize_kmer and nb_attn_fwd")}
     del sets, host, outs
     return res
 

@@ -28,8 +28,8 @@
 // key row; they also stage dK (first) and dV (second) of an item in its K/V
 // buffer after the next item's first chunk (so the wait for the item's last
 // products overlaps that chunk's arithmetic);
-// warpgroup 3: dQ warps, thread = query row, stage dQ_c in shared memory and
-// reduce it into global memory.  All waits are bounded (see sm100.cuh).
+// warpgroup 3: dQ warps, thread = query row; each warp stages its 32 rows of
+// dQ_c in its own shared-memory box and reduce-adds them into global memory.  All waits are bounded (see sm100.cuh).
 #include <math.h>
 
 #include "nb_internal.h"
@@ -51,7 +51,8 @@ template <int D>
 struct Cfg {
   static_assert(D == 64, "this kernel is the d = 64 one");
   // K/V tiles double-buffered, three Q/dO stages; P^T kept in TMEM (64 spare
-  // columns) as the A operand of dV; dQ staged through one 128 x 32 fp32 box,
+  // columns) as the A operand of dV; dQ staged through one 128 x 32 fp32 area
+  // (a 32 x 32 box per dQ warp),
   // so a chunk's Q/dO buffer is free as soon as its gradient products complete.
   static constexpr int NKV = 2;  // K/V tile buffers
   static constexpr int NS = 3;   // Q/dO chunk stages
@@ -60,7 +61,7 @@ struct Cfg {
   static constexpr int oK = 0;                   // buffer i: K at oK + 2 i kTile, V after it
   static constexpr int oQ = NKV * 2 * kTile;     // stage s: Q at oQ + 2 s kTile, dO after it
   static constexpr int oDS = oQ + NS * 2 * kTile;  // dS^T tile
-  static constexpr int oStg = oDS + kPT;  // dQ staging box (one 128 x 32 fp32 box)
+  static constexpr int oStg = oDS + kPT;  // dQ staging: warp w's 32 x 32 fp32 box at + 4 KB w
   // The dK/dV epilogue of an item is deferred past the next item's first
   // chunk (the next item's K/V tile has a buffer of its own).
   static constexpr int oLD = oStg + kSlab;  // stage s: -lse log2e, D
@@ -69,7 +70,7 @@ struct Cfg {
                        bQDFree = bQDFull + NS, bSDPFull = bQDFree + NS, bSDPFree = bSDPFull + 1,
                        bPDSFull = bSDPFree + 1, bPDSFree = bPDSFull + 1, bDQFull = bPDSFree + 1,
                        bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
-                       bStg = bDKVFree + 1, bStgFree = bStg + 1, bOutFull = bStgFree + 1,
+                       bOutFull = bDKVFree + 1,
                        bDone = bOutFull + NKV,
                        nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
@@ -135,7 +136,7 @@ __device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int 
 
 enum : int { kErrKVFree = 0x31, kErrQDFree, kErrKVFull, kErrQDFull, kErrSDPFree, kErrDQFree,
              kErrPDSFull, kErrDKVFree, kErrGQD, kErrSDPFull, kErrPDSFree, kErrDKVFull,
-             kErrDQFull, kErrDone, kErrStg, kErrStgFree, kErrOutFull };
+             kErrDQFull, kErrDone, kErrOutFull };
 
 template <int D>
 __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tk,
@@ -475,16 +476,17 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
   return 0;
 }
 
-// dQ warps: thread = query row r of the chunk.
+// dQ warps: thread = query row of the chunk (warp w: rows 32 w .. 32 w + 31).
+// Each warp stages its 32 rows of a 32-column box in its own 4 KB of the
+// staging area and reduce-adds them with its own TMA bulk reduce, so the four
+// warps never wait for one another.
 template <int D>
 __device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
                         uint32_t tmem, int wq, int lane, const CUtensorMap* tdq) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
-  const int r = wq * 32 + lane;
   const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-  const bool leader = threadIdx.x == 12 * 32;
   auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
   int g = 0;
   for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
@@ -496,7 +498,7 @@ __device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint8_
       const int q0 = (x.I0 + 4 * c) * kBlock;
       if (!all_ok(mbar_wait(bar + 8 * C::bDQFull, G & 1))) return kErrDQFull;
       tc_fence_after();
-      // dQ_c through the staging box, one 32-column box per pass; the row is read
+      // dQ_c through the warp's staging box, one 32-column box per pass; the row is read
       // from TMEM 64 columns at a time and its TMEM released after the last read
       uint8_t* stg = gbase + C::oStg;
 #pragma unroll
@@ -513,28 +515,27 @@ __device__ int dq_warps(const Params& p, const Sched& sch, uint32_t base, uint8_
         }
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
-          const int j = 2 * grp + jj;      // box (32 columns) within the row
-          const int k = G * (D / 32) + j;  // global pass index
-          if (!all_ok(mbar_wait(bar + 8 * C::bStgFree, (k & 1) ^ 1))) return kErrStgFree;
+          const int j = 2 * grp + jj;  // 32-column box within the row
+          // this warp's 32 rows go through its own 4 KB box and its own reduce-add
+          if (lane == 0) bulk_wait_read0();  // the box's previous reduce-add has read it
+          __syncwarp();
+          uint8_t* box = stg + wq * 4096;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<float4*>(stg + r * 128 + ((u ^ (r & 7)) << 4)) =
+            *reinterpret_cast<float4*>(box + lane * 128 + ((u ^ (lane & 7)) << 4)) =
                 make_float4(v[jj][4 * u], v[jj][4 * u + 1], v[jj][4 * u + 2], v[jj][4 * u + 3]);
           fence_proxy_async_smem();
-          mbar_arrive(bar + 8 * C::bStg);  // this thread's row of the box is written
-          if (leader) {
-            if (!mbar_wait(bar + 8 * C::bStg, k & 1)) return kErrStg;
-            tma_reduce_add_3d(tdq, base + C::oStg, 32 * j, q0, bh);
+          __syncwarp();
+          if (lane == 0 && q0 + 32 * wq < a.n) {
+            tma_reduce_add_3d(tdq, base + C::oStg + wq * 4096, 32 * j, q0 + 32 * wq, bh);
             bulk_commit();
-            bulk_wait_read0();
-            mbar_arrive(bar + 8 * C::bStgFree);
           }
         }
       }
     }
     g += x.nch;
   }
-  if (leader) bulk_wait_all0();  // the last reduce-adds have read shared memory and landed
+  if (lane == 0) bulk_wait_all0();  // the last reduce-adds have read shared memory and landed
   return 0;
 }
 
@@ -569,8 +570,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar + 8 * C::bDQFree, 128);
     mbar_init(bar + 8 * C::bDKVFull, 1);
     mbar_init(bar + 8 * C::bDKVFree, 256);
-    mbar_init(bar + 8 * C::bStg, 128);
-    mbar_init(bar + 8 * C::bStgFree, 1);
     for (int i = 0; i < C::NKV; ++i) mbar_init(bar + 8 * (C::bOutFull + i), 256);
     mbar_init(bar + 8 * C::bDone, 2);  // one commit per MMA-issuing thread
     fence_barrier_init();
@@ -648,7 +647,7 @@ cudaError_t launch(const AttnArgs& a, int64_t rows, cudaStream_t stream) {
       !make_tmap_bf16_rows(&tv, a.v, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tq, a.q, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tdo, a.dout, D, a.n, heads_total, kRows) ||
-      !make_tmap_rows(&tdq, p.ws.dqacc, true, D, a.n, heads_total, 32, kRows) ||
+      !make_tmap_rows(&tdq, p.ws.dqacc, true, D, a.n, heads_total, 32, 32) ||
       !make_tmap_bf16_rows(&tdk, a.dk, D, a.n, heads_total, kRows) ||
       !make_tmap_bf16_rows(&tdv, a.dv, D, a.n, heads_total, kRows))
     return cudaErrorInvalidValue;

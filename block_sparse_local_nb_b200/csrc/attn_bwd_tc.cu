@@ -29,7 +29,8 @@
 // buffer after the next item's first chunk (so the wait for the item's last
 // products overlaps that chunk's arithmetic);
 // warpgroup 3: dQ warps, thread = query row; each warp stages its 32 rows of
-// dQ_c in its own shared-memory box and reduce-adds them into global memory.  All waits are bounded (see sm100.cuh).
+// dQ_c in its own shared-memory box and reduce-adds them into global memory.
+// All waits are bounded (see sm100.cuh).
 #include <math.h>
 
 #include "nb_internal.h"

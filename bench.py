@@ -528,6 +528,43 @@ def time_attention(w, args, dev, rank, world, with_e2e, steps, warmup):
     return res
 
 
+def time_host_link(nbytes=1 << 30, reps=5):
+    """Host link bandwidth with pinned buffers: host->device alone, device->host
+    alone, and both at once on two streams (GB/s per direction, CUDA events)."""
+    import torch
+
+    h_src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    h_dst = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d_a = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    d_b = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def run(h2d, d2h):
+        main = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for timed in (False, True):
+            torch.cuda.synchronize()
+            e0.record(main)
+            s_in.wait_stream(main)
+            s_out.wait_stream(main)
+            for _ in range(reps if timed else 2):
+                if h2d:
+                    with torch.cuda.stream(s_in):
+                        d_a.copy_(h_src, non_blocking=True)
+                if d2h:
+                    with torch.cuda.stream(s_out):
+                        h_dst.copy_(d_b, non_blocking=True)
+            main.wait_stream(s_in)
+            main.wait_stream(s_out)
+            e1.record(main)
+        torch.cuda.synchronize()
+        return nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9
+
+    return {"metric": "host link bandwidth, pinned cudaMemcpyAsync", "unit": "GB/s per direction",
+            "bytes_per_copy": nbytes, "h2d": run(True, False), "d2h": run(False, True),
+            "both_at_once": run(True, True)}
+
+
 def attention_line(res, peaks, peak_kind, world):
     """The JSON fields of one attention workload's measurement."""
     w, alg = res["w"], res["alg"]
@@ -702,6 +739,9 @@ def main():
     ap.add_argument("--no-sub", action="store_true", help="headline workload only")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end (host buffers) measurement, for quick comparisons")
+    ap.add_argument("--link", action="store_true",
+                    help="only measure the host link: pinned copies host->device, "
+                         "device->host and both at once (the end-to-end ceiling)")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override n of a full-length workload (a smaller case of the same "
                          "shape, e.g. for profiling)")
@@ -715,6 +755,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.link:
+        if rank == 0:
+            print(json.dumps(time_host_link()), flush=True)
+        return
     if args.workload == "dna_batch_ids":
         if args.impl == "native" and rank == 0:
             run_batch_ids_workload(args)

@@ -41,7 +41,8 @@ def _device_step(q, k, v, do, lengths, R, causal=False):
 # chunks of a few heads of one row (a short last chunk); more chunks than
 # workspace slots; too few slices, so each is cut into windows with 2R blocks
 # of context (8 windows of 8 blocks at R = 2; 3 windows of 43 blocks at R = 9,
-# lengths ending inside a window's context and inside an owned range)
+# lengths ending inside a window's context and inside an owned range; 32
+# windows of a 65536-token sequence)
 CASES = [
     (1, 1, 288, 2, [200], False),
     (16, 2, 96, 1, [96, 1, 33, 64] * 4, False),
@@ -49,6 +50,8 @@ CASES = [
     (3, 5, 288, 9, [288, 0, 131], False),
     (1, 2, 2048, 2, [1900], True),
     (2, 1, 4096, 9, [4096, 2790], True),
+    # 32 windows of 64 blocks, the last ones all padding
+    (1, 1, 65536, 1, [60000], True),
 ]
 
 

@@ -91,14 +91,13 @@ struct Item {
   int b, h, tile, L, I0, nch;
 };
 
-__device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int tile) {
+__device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int tile, int L) {
   const AttnArgs& a = p.a;
   Item x;
   x.b = b;
   x.h = h;
   x.tile = tile;
-  int L = a.lengths ? a.lengths[x.b] : a.n;
-  x.L = min(max(L, 0), a.n);
+  x.L = L;  // clamped to [0, n]
   const int nb = a.n / kBlock;
   x.I0 = 0;
   x.nch = 0;
@@ -114,14 +113,15 @@ __device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int ti
 __device__ __forceinline__ Item decode(const Params& p, int it) {
   const int bh = it / p.ntiles;
   const int b = bh / p.a.heads;
-  return decode_bht(p, b, bh - b * p.a.heads, it - bh * p.ntiles);
+  const int L = p.a.lengths ? p.a.lengths[b] : p.a.n;
+  return decode_bht(p, b, bh - b * p.a.heads, it - bh * p.ntiles, min(max(L, 0), p.a.n));
 }
 
 __device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int k) {
   if (!s.balanced) return decode(p, k);
   int b, h, tile;
   sched_nonempty(s, p.a.batch, p.a.heads, k, b, h, tile);
-  return decode_bht(p, b, h, tile);
+  return decode_bht(p, b, h, tile, sched_length(s, p.a, b));
 }
 
 enum : int { kErrKVFree = 0x51, kErrQDFree, kErrKVFull, kErrQDFull, kErrSDPFree, kErrDQFree,
@@ -403,7 +403,7 @@ __device__ int grad_warps(const Params& p, const Sched& sch, uint32_t base, uint
     for (int e = blockIdx.x; e < p.items - sch.count; e += gridDim.x) {
       int b, h, tile;
       sched_empty(sch, a.batch, a.heads, p.ntiles, e, b, h, tile);
-      zero_tile(decode_bht(p, b, h, tile));
+      zero_tile(decode_bht(p, b, h, tile, sched_length(sch, a, b)));
     }
   }
   return 0;

@@ -12,18 +12,18 @@
 // walks the items; consecutive CTAs take neighbouring tiles at the same time,
 // so the key/value blocks their windows share are served from L2.
 //
-// Warp roles (352 threads):
+// Warp roles (512 threads, four warpgroups with reallocated registers):
 //   warp 0     TMA producer: Q tile, then K and V chunks, into 128-byte
 //              swizzled shared memory (3-D tensor maps; rows outside [0, n)
 //              are zero-filled by TMA and masked).
 //   warp 1     TMEM owner and S issuer (one thread):
 //                S_c = Q K_c^T   (M 128, N 128, K d)   -> TMEM, two buffers
-//   warp 10    P V issuer (one thread):
+//   warp 2     P V issuer (one thread):
 //                O_h += P_c,h V_c,h  (M 128, N d, K 64; P read from TMEM)
 //              Two issuing threads keep the tensor pipe fed: a lone thread
 //              issuing both streams serialises every wait and commit with
 //              the MMAs.  S_{c+1} is in flight while chunk c's softmax runs.
-//   warps 2-9  softmax, two groups of four warps; thread (r, half) owns row r
+//   warps 4-11 softmax, two groups of four warps; thread (r, half) owns row r
 //              (TMEM lane r) and 64 of the chunk's 128 key columns.  Per chunk
 //              it reads its 64 scores, masks keys outside its query block's
 //              band or past the length, updates its own running max and sum
@@ -31,12 +31,15 @@
 //              the scores it has read.  Each half keeps its own running output
 //              O_h in TMEM; it is rescaled (load, multiply, store) only when
 //              that half's max grows by more than 2^8, otherwise the stale max
-//              is kept (P <= 2^8, exact after the final division).
-//              Epilogue (deferred past the next item's first chunk): the
-//              halves exchange (m, l) through shared memory and combine
+//              is kept (P <= 2^8, exact after the final division).  At the end
+//              of a tile each half hands its (m, l) of the row to the epilogue
+//              warps through shared memory and goes on to the next tile.
+//   warps 12-15 epilogue, thread = row: combine the halves
 //              O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / l, lse = M + log l;
 //              the bf16 tile is staged in swizzled shared memory and written
-//              by one TMA tensor store (coalesced, asynchronous).
+//              by one TMA tensor store (coalesced, asynchronous).  The O
+//              accumulators are double-buffered at d = 64, so the next tile's
+//              P V products do not wait for this.
 // Every mbarrier wait is bounded; on a timeout the kernel records an error
 // code in the caller-visible error word and tears down (frees TMEM) instead
 // of hanging.
@@ -51,7 +54,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 512;
 constexpr int kRows = 128;   // query rows per tile
 constexpr int kChunk = 128;  // keys per chunk
 constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 64 bf16
@@ -75,10 +78,11 @@ struct Cfg {
   static constexpr int bQFull = 0, bQFree = bQFull + NQ, bKVFull = bQFree + NQ,
                        bKVFree = bKVFull + NKV, bSFull = bKVFree + NKV, bSFree = bSFull + 2,
                        bPFull = bSFree + 2, bPVDone = bPFull + 4, bOFull = bPVDone + 4,
-                       bOFree = bOFull + 2 * NOB, bXSum = bOFree + 2 * NOB, bDone = bXSum + 2,
-                       nBar = bDone + 1;
+                       bOFree = bOFull + 2 * NOB, bXFull = bOFree + 2 * NOB, bXFree = bXFull + 2,
+                       bDone = bXFree + 2, nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
-  // per-tile exchange of the halves' running max and sum: [parity][half][m, l][row] fp32
+  // per-tile hand-off of the halves' running max and sum to the epilogue warps:
+  // [parity][half][m, l][row] fp32
   static constexpr int oXSum = oSlot + 16;
   static constexpr int oSched = oXSum + 2 * 2 * 2 * 128 * 4;  // work-order prefix table
   static constexpr int kSmem = oSched + kSchedBytes + 1024;  // + slack for 1024-byte alignment
@@ -90,6 +94,12 @@ struct Cfg {
   __device__ static constexpr uint32_t tP(int sb, int h) { return tS + sb * kChunk + 64 * h; }
   // O accumulator of half h, buffer ob
   __device__ static constexpr uint32_t tO(int h, int ob) { return 256 + (h * NOB + ob) * D; }
+  // registers per thread after reallocation: TMA/MMA warpgroup, each softmax
+  // warpgroup, epilogue warpgroup (the 16 warps share the 64K-register file)
+  static constexpr int kRegsCtl = 56;
+  static constexpr int kRegsSoft = 168;
+  static constexpr int kRegsEpi = 120;
+  static_assert(128 * (kRegsCtl + 2 * kRegsSoft + kRegsEpi) <= 65536, "register budget");
 };
 
 struct Params {
@@ -102,14 +112,13 @@ struct Item {
   int b, h, tile, L, J0, nch;
 };
 
-__device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int tile) {
+__device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int tile, int L) {
   const AttnArgs& a = p.a;
   Item x;
   x.b = b;
   x.h = h;
   x.tile = tile;
-  int L = a.lengths ? a.lengths[x.b] : a.n;
-  x.L = min(max(L, 0), a.n);
+  x.L = L;  // clamped to [0, n]
   const int nb = a.n / kBlock;
   x.J0 = 0;
   x.nch = 0;
@@ -126,7 +135,8 @@ __device__ __forceinline__ Item decode_bht(const Params& p, int b, int h, int ti
 __device__ __forceinline__ Item decode(const Params& p, int it) {
   const int bh = it / p.ntiles;
   const int b = bh / p.a.heads;
-  return decode_bht(p, b, bh - b * p.a.heads, it - bh * p.ntiles);
+  const int L = p.a.lengths ? p.a.lengths[b] : p.a.n;
+  return decode_bht(p, b, bh - b * p.a.heads, it - bh * p.ntiles, min(max(L, 0), p.a.n));
 }
 
 // Item k of the first pass (non-empty tiles when balanced, else every tile).
@@ -134,12 +144,12 @@ __device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int 
   if (!s.balanced) return decode(p, k);
   int b, h, tile;
   sched_nonempty(s, p.a.batch, p.a.heads, k, b, h, tile);
-  return decode_bht(p, b, h, tile);
+  return decode_bht(p, b, h, tile, sched_length(s, p.a, b));
 }
 
 // error codes: 0x10 + site
 enum : int { kErrQFree = 0x11, kErrKVFree, kErrQFull, kErrKVFull, kErrSFree, kErrOFree, kErrPFull,
-             kErrSFull, kErrPPrev = 0x1a, kErrOFull, kErrDone, kErrXSum = 0x1e };
+             kErrSFull, kErrPPrev = 0x1a, kErrOFull, kErrDone, kErrXFull = 0x1e, kErrXFree };
 
 template <int D>
 __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tq,
@@ -253,8 +263,8 @@ __device__ int pv_issuer(const Params& p, const Sched& sch, uint32_t base, uint3
 }
 
 template <int D, bool kCausal>
-__device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
-                                uint32_t tmem, int wq, int hf, int lane, const CUtensorMap* to) {
+__device__ int softmax_warps(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
+                             uint32_t tmem, int wq, int hf, int lane) {
   using C = Cfg<D>;
   const AttnArgs& a = p.a;
   const uint32_t bar = base + C::oBar;
@@ -264,81 +274,6 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
   const float sl2 = a.scale * kLog2e;
   float* xs = reinterpret_cast<float*>(gbase + C::oXSum);
   auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
-  // An item's epilogue runs after the next item's first chunk, so the wait for
-  // its last P V product overlaps that chunk's softmax.
-  struct Epi {
-    bool valid;
-    int tc, bh, tile;
-    int64_t row;  // global row index of this thread's query (bh * n + q)
-    bool in_range;
-    float m, l;   // this half's running max (base 2) and sum
-  } pend = {false, 0, 0, 0, 0, false, 0.f, 0.f};
-  // One thread stores the staged output tile with TMA; before the staging
-  // buffer is written again it waits until that store has read it.
-  const bool leader = wq == 2 && hf == 0 && lane == 0;
-  uint8_t* stg = gbase + C::oStg;
-  // Combine the halves: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)).
-  auto epilogue = [&](const Epi& x) -> int {
-    const int ob = x.tc % C::NOB, par = x.tc & 1;
-    if (leader) bulk_wait_read0();  // the previous tile's store is done with the staging
-    xs[((par * 2 + hf) * 2 + 0) * 128 + r] = x.m;
-    xs[((par * 2 + hf) * 2 + 1) * 128 + r] = x.l;
-    mbar_arrive(bar + 8 * (C::bXSum + par));
-    if (!all_ok(mbar_wait(bar + 8 * (C::bXSum + par), (x.tc >> 1) & 1))) return kErrXSum;
-    const float mo = xs[((par * 2 + (hf ^ 1)) * 2 + 0) * 128 + r];
-    const float lo = xs[((par * 2 + (hf ^ 1)) * 2 + 1) * 128 + r];
-    const float M = fmaxf(x.m, mo);
-    const float fs = x.m == -INFINITY ? 0.f : ex2_approx(x.m - M);
-    const float fo = mo == -INFINITY ? 0.f : ex2_approx(mo - M);
-    const float L = x.l * fs + lo * fo;
-    const float f0 = hf == 0 ? fs : fo, f1 = hf == 0 ? fo : fs;  // factors of O_0 and O_1
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      if (!all_ok(mbar_wait(bar + 8 * (C::bOFull + h * C::NOB + ob), (x.tc / C::NOB) & 1)))
-        return kErrOFull;
-    tc_fence_after();
-    float o0[D / 64][32], o1[D / 64][32];  // this half's D/2 output columns of O_0 and O_1
-#pragma unroll
-    for (int j = 0; j < D / 64; ++j) {
-      tmem_ld32(trow + C::tO(0, ob) + hf * (D / 2) + 32 * j, o0[j]);
-      tmem_ld32(trow + C::tO(1, ob) + hf * (D / 2) + 32 * j, o1[j]);
-    }
-    tmem_wait_ld();
-#pragma unroll
-    for (int j = 0; j < D / 64; ++j) {
-      reg_fence(o0[j]);
-      reg_fence(o1[j]);
-    }
-    tc_fence_before();
-    mbar_arrive(bar + 8 * (C::bOFree + 0 * C::NOB + ob));
-    mbar_arrive(bar + 8 * (C::bOFree + 1 * C::NOB + ob));
-    const bool has = L > 0.f;  // padding rows and rows without a visible key: 0
-    const float inv = has ? 1.f / L : 0.f;
-    const float g0 = f0 * inv, g1 = f1 * inv;
-    // this half's D / 2 columns = D / 16 chunks of 16 bytes in the swizzled staging
-#pragma unroll
-    for (int j = 0; j < D / 64; ++j) {
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        float w8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) w8[i] = fmaf(o0[j][8 * v + i], g0, o1[j][8 * v + i] * g1);
-        const int gc = hf * (D / 16) + 4 * j + v;  // chunk index within the output row
-        *reinterpret_cast<uint4*>(stg + (gc >> 3) * kSlab + r * 128 + (((gc & 7) ^ (r & 7)) << 4)) =
-            make_uint4(pack_bf16(w8[0], w8[1]), pack_bf16(w8[2], w8[3]), pack_bf16(w8[4], w8[5]),
-                       pack_bf16(w8[6], w8[7]));
-      }
-    }
-    if (x.in_range && a.lse && hf == 0) a.lse[x.row] = has ? (M + log2f(L)) * kLn2 : -INFINITY;
-    fence_proxy_async_smem();
-    named_barrier(1, 256);  // the whole tile is staged
-    if (leader) {
-#pragma unroll
-      for (int s = 0; s < D / 64; ++s) tma_store_3d(to, base + C::oStg + s * kSlab, s * 64, x.tile * kRows, x.bh);
-      bulk_commit();
-    }
-    return 0;
-  };
   // a tile entirely past its sequence's length: O = 0, lse = -inf
   // (the tile's rows are contiguous: the 256 threads store it as one coalesced run)
   auto zero_tile = [&](const Item& x) {
@@ -349,10 +284,9 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
     for (int i = hf * 128 + r; i < rows * (D / 8); i += 256) out[i] = make_uint4(0, 0, 0, 0);
     if (a.lse && hf == 0 && r < rows) a.lse[row0 + r] = -INFINITY;
   };
-  int g = 0, tc = 0, e = 0;
+  int g = 0, tc = 0;
   for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
     const Item x = sched_item(p, sch, it);
-    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
     const int q = x.tile * kRows + r;
     if (x.nch == 0) {  // the whole tile is padding
       zero_tile(x);
@@ -452,24 +386,102 @@ __device__ int softmax_epilogue(const Params& p, const Sched& sch, uint32_t base
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar + 8 * (C::bPFull + 2 * sb + hf));
-      if (c == 0 && pend.valid) {  // the previous item's epilogue, deferred past this chunk
-        if ((e = epilogue(pend))) return e;
-        pend.valid = false;
-      }
     }
-    pend = {true, tc, static_cast<int>(bh), x.tile, bh * a.n + q, q < a.n, m_used, l};
+    // hand this half's (m, l) of the row to the epilogue warps
+    const int par = tc & 1;
+    if (!all_ok(mbar_wait(bar + 8 * (C::bXFree + par), ((tc >> 1) & 1) ^ 1))) return kErrXFree;
+    xs[((par * 2 + hf) * 2 + 0) * 128 + r] = m_used;
+    xs[((par * 2 + hf) * 2 + 1) * 128 + r] = l;
+    mbar_arrive(bar + 8 * (C::bXFull + par));
     g += x.nch;
     ++tc;
   }
-  if (pend.valid && (e = epilogue(pend))) return e;
-  if (leader) bulk_wait_all0();  // the last tile's store has landed before the CTA exits
   if (sch.balanced) {  // second pass: the empty tiles, listed directly
     for (int e = blockIdx.x; e < p.items - sch.count; e += gridDim.x) {
       int b, h, tile;
       sched_empty(sch, a.batch, a.heads, p.ntiles, e, b, h, tile);
-      zero_tile(decode_bht(p, b, h, tile));
+      zero_tile(decode_bht(p, b, h, tile, sched_length(sch, a, b)));
     }
   }
+  return 0;
+}
+
+// Epilogue warps (one warpgroup, thread = tile row r): per tile, combine the
+// halves O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / l, l = l_0 2^(m_0 - M) +
+// l_1 2^(m_1 - M), lse = M + log l; stage the bf16 tile in swizzled shared
+// memory and write it with one TMA tensor store.  Off the softmax warps' path:
+// they hand over (m, l) and move on to the next tile.
+template <int D>
+__device__ int epi_warps(const Params& p, const Sched& sch, uint32_t base, uint8_t* gbase,
+                         uint32_t tmem, int wq, int lane, const CUtensorMap* to) {
+  using C = Cfg<D>;
+  const AttnArgs& a = p.a;
+  const uint32_t bar = base + C::oBar;
+  const int r = wq * 32 + lane;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const float* xs = reinterpret_cast<const float*>(gbase + C::oXSum);
+  uint8_t* stg = gbase + C::oStg;
+  const bool leader = r == 0;
+  auto all_ok = [](bool ok) { return __all_sync(0xffffffffu, ok); };
+  int tc = 0;
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
+    if (x.nch == 0) continue;
+    const int64_t bh = static_cast<int64_t>(x.b) * a.heads + x.h;
+    const int ob = tc % C::NOB, par = tc & 1;
+    if (!all_ok(mbar_wait(bar + 8 * (C::bXFull + par), (tc >> 1) & 1))) return kErrXFull;
+    const float m0 = xs[((par * 2 + 0) * 2 + 0) * 128 + r], l0 = xs[((par * 2 + 0) * 2 + 1) * 128 + r];
+    const float m1 = xs[((par * 2 + 1) * 2 + 0) * 128 + r], l1 = xs[((par * 2 + 1) * 2 + 1) * 128 + r];
+    mbar_arrive(bar + 8 * (C::bXFree + par));
+    const float M = fmaxf(m0, m1);
+    const float f0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M);
+    const float f1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - M);
+    const float L = l0 * f0 + l1 * f1;
+    const bool has = L > 0.f;  // padding rows and rows without a visible key: 0
+    const float inv = has ? 1.f / L : 0.f;
+    const float g0 = f0 * inv, g1 = f1 * inv;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (!all_ok(mbar_wait(bar + 8 * (C::bOFull + h * C::NOB + ob), (tc / C::NOB) & 1)))
+        return kErrOFull;
+    tc_fence_after();
+    if (leader) bulk_wait_read0();  // the previous tile's store is done with the staging
+    named_barrier(2, 128);
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) {  // 32 output columns at a time
+      float o0[32], o1[32];
+      tmem_ld32(trow + C::tO(0, ob) + 32 * j, o0);
+      tmem_ld32(trow + C::tO(1, ob) + 32 * j, o1);
+      tmem_wait_ld();
+      reg_fence(o0);
+      reg_fence(o1);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        float w8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w8[i] = fmaf(o0[8 * v + i], g0, o1[8 * v + i] * g1);
+        const int gc = 4 * j + v;  // 16-byte chunk index within the output row
+        *reinterpret_cast<uint4*>(stg + (gc >> 3) * kSlab + r * 128 + (((gc & 7) ^ (r & 7)) << 4)) =
+            make_uint4(pack_bf16(w8[0], w8[1]), pack_bf16(w8[2], w8[3]), pack_bf16(w8[4], w8[5]),
+                       pack_bf16(w8[6], w8[7]));
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(bar + 8 * (C::bOFree + 0 * C::NOB + ob));
+    mbar_arrive(bar + 8 * (C::bOFree + 1 * C::NOB + ob));
+    const int q = x.tile * kRows + r;
+    if (q < a.n && a.lse) a.lse[bh * a.n + q] = has ? (M + log2f(L)) * kLn2 : -INFINITY;
+    fence_proxy_async_smem();
+    named_barrier(1, 128);  // the whole tile is staged
+    if (leader) {
+#pragma unroll
+      for (int s = 0; s < D / 64; ++s)
+        tma_store_3d(to, base + C::oStg + s * kSlab, s * 64, x.tile * kRows, static_cast<int>(bh));
+      bulk_commit();
+    }
+    ++tc;
+  }
+  if (leader) bulk_wait_all0();  // the last tile's store has landed before the CTA exits
   return 0;
 }
 
@@ -498,7 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + 8 * (C::bSFull + i), 1);
       mbar_init(bar + 8 * (C::bSFree + i), 1);
-      mbar_init(bar + 8 * (C::bXSum + i), 256);
+      mbar_init(bar + 8 * (C::bXFull + i), 256);
+      mbar_init(bar + 8 * (C::bXFree + i), 128);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(bar + 8 * (C::bPFull + i), 128);
@@ -506,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2 * C::NOB; ++i) {
       mbar_init(bar + 8 * (C::bOFull + i), 1);
-      mbar_init(bar + 8 * (C::bOFree + i), 256);
+      mbar_init(bar + 8 * (C::bOFree + i), 128);
     }
     mbar_init(bar + 8 * C::bDone, 2);  // one commit per MMA-issuing thread
     fence_barrier_init();
@@ -532,21 +545,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Sched sch = sched_view(reinterpret_cast<const int*>(gbase + C::oSched), p.a, p.items);
 
   int err = 0;
-  if (warp == 0) {
-    if (lane == 0) err = producer<D>(p, sch, base, &tq, &tk, &tv);
-  } else if (warp == 1) {
-    if (lane == 0) err = s_issuer<D>(p, sch, base, tmem);
-  } else if (warp == 10) {
-    if (lane == 0) err = pv_issuer<D>(p, sch, base, tmem);
+  if (warp < 4) {
+    regs_dec<C::kRegsCtl>();
+    if (warp == 0 && lane == 0) err = producer<D>(p, sch, base, &tq, &tk, &tv);
+    if (warp == 1 && lane == 0) err = s_issuer<D>(p, sch, base, tmem);
+    if (warp == 2 && lane == 0) err = pv_issuer<D>(p, sch, base, tmem);
+  } else if (warp < 12) {
+    regs_inc<C::kRegsSoft>();
+    err = softmax_warps<D, kCausal>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
   } else {
-    err = softmax_epilogue<D, kCausal>(p, sch, base, gbase, tmem, warp & 3, (warp - 2) >> 2, lane,
-                                       &to);
+    regs_dec<C::kRegsEpi>();
+    err = epi_warps<D>(p, sch, base, gbase, tmem, warp & 3, lane, &to);
   }
   if (err) record_error(p.a.err, err);
 
   pdl_trigger();  // this CTA's work is issued: the next kernel may start launching
   __syncthreads();
-  if (warp == 10 && lane == 0) mma_commit(bar + 8 * C::bDone);
+  if (warp == 2 && lane == 0) mma_commit(bar + 8 * C::bDone);
   if (warp == 1) {
     if (lane == 0) {  // every tensor-core operation of this CTA has completed
       mma_commit(bar + 8 * C::bDone);

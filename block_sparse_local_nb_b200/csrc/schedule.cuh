@@ -9,8 +9,10 @@
 // is full length).  The list is implicit: a
 // prefix table over sequences, pre[b] = number of non-empty tiles (all heads)
 // of sequences before b, built once per CTA in shared memory and searched per
-// item.  Batches larger than kMaxSchedBatch fall back to a round-robin over all
-// tiles.
+// item.  The clamped lengths sit beside it, so that decoding an item reads
+// shared memory only (a global load there would stall every role of the CTA
+// at each item boundary).  Batches larger than kMaxSchedBatch fall back to a
+// round-robin over all tiles, with the lengths read from global memory.
 #pragma once
 
 #include "nb_internal.h"
@@ -18,9 +20,11 @@
 namespace nb {
 
 constexpr int kMaxSchedBatch = 1024;
-constexpr int kSchedBytes = (kMaxSchedBatch + 1) * 4;
+// pre[0..batch], then the clamped lengths len[0..batch) from pre + kMaxSchedBatch + 1
+constexpr int kSchedBytes = (2 * kMaxSchedBatch + 1) * 4;
 
-// Warp-cooperative: fills pre[0..batch] (call with one full warp, then sync the CTA).
+// Warp-cooperative: fills pre[0..batch] and len[0..batch) (call with one full
+// warp, then sync the CTA).
 __device__ __forceinline__ void sched_build(int* pre, const AttnArgs& a, int rows_per_tile,
                                             int lane) {
   if (a.batch > kMaxSchedBatch) return;
@@ -31,6 +35,7 @@ __device__ __forceinline__ void sched_build(int* pre, const AttnArgs& a, int row
     if (b < a.batch) {
       int L = a.lengths ? a.lengths[b] : a.n;
       L = min(max(L, 0), a.n);
+      pre[kMaxSchedBatch + 1 + b] = L;
       v = a.heads * ((L + rows_per_tile - 1) / rows_per_tile);
     }
 #pragma unroll
@@ -46,16 +51,25 @@ __device__ __forceinline__ void sched_build(int* pre, const AttnArgs& a, int row
 
 struct Sched {
   const int* pre;
-  bool balanced;  // walk the non-empty list (else every tile, round-robin)
-  int count;      // items of the first pass
+  const int* len;  // clamped lengths (balanced only)
+  bool balanced;   // walk the non-empty list (else every tile, round-robin)
+  int count;       // items of the first pass
 };
 
 __device__ __forceinline__ Sched sched_view(const int* pre, const AttnArgs& a, int all_items) {
   Sched s;
   s.pre = pre;
+  s.len = pre + kMaxSchedBatch + 1;
   s.balanced = a.batch <= kMaxSchedBatch;
   s.count = s.balanced ? pre[a.batch] : all_items;
   return s;
+}
+
+// Length of sequence b clamped to [0, n].
+__device__ __forceinline__ int sched_length(const Sched& s, const AttnArgs& a, int b) {
+  if (s.balanced) return s.len[b];
+  const int L = a.lengths ? a.lengths[b] : a.n;
+  return min(max(L, 0), a.n);
 }
 
 // (sequence, head, tile) of item k of the non-empty list.

@@ -17,12 +17,14 @@
 //              swizzled shared memory (3-D tensor maps; rows outside [0, n)
 //              are zero-filled by TMA and masked).
 //   warp 1     TMEM owner and S issuer (one thread):
-//                S_c = Q K_c^T   (M 128, N 128, K d)   -> TMEM, two buffers
+//                S_c = Q K_c^T   (M 128, N 128, K d)   -> TMEM, three buffers at
+//                d = 64 (S of chunks c + 1 and c + 2 in flight while chunk c's
+//                softmax runs), two at d = 128
 //   warp 2     P V issuer (one thread):
 //                O_h += P_c,h V_c,h  (M 128, N d, K 64; P read from TMEM)
 //              Two issuing threads keep the tensor pipe fed: a lone thread
 //              issuing both streams serialises every wait and commit with
-//              the MMAs.  S_{c+1} is in flight while chunk c's softmax runs.
+//              the MMAs.
 //   warps 4-11 softmax, two groups of four warps; thread (r, half) owns row r
 //              (TMEM lane r) and 64 of the chunk's 128 key columns.  Per chunk
 //              it reads its 64 scores, masks keys outside its query block's
@@ -37,9 +39,9 @@
 //   warps 12-15 epilogue, thread = row: combine the halves
 //              O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / l, lse = M + log l;
 //              the bf16 tile is staged in swizzled shared memory and written
-//              by one TMA tensor store (coalesced, asynchronous).  The O
-//              accumulators are double-buffered at d = 64, so the next tile's
-//              P V products do not wait for this.
+//              by one TMA tensor store (coalesced, asynchronous).  The next
+//              tile's first P V product waits until these warps have read O;
+//              the softmax of that tile's first chunks does not.
 // Every mbarrier wait is bounded; on a timeout the kernel records an error
 // code in the caller-visible error word and tears down (frees TMEM) instead
 // of hanging.
@@ -66,7 +68,8 @@ template <int D>
 struct Cfg {
   static constexpr int NQ = D == 64 ? 2 : 1;   // Q tile buffers
   static constexpr int NKV = D == 64 ? 3 : 2;  // K/V chunk stages
-  static constexpr int NOB = D == 64 ? 2 : 1;  // O accumulators per half (tiles in flight)
+  static constexpr int NSB = D == 64 ? 3 : 2;  // S buffers
+  static constexpr int NOB = 1;  // O accumulators per half (tiles in flight)
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kKBytes = kChunk * D * 2;
   static constexpr int oQ = 0;
@@ -76,8 +79,8 @@ struct Cfg {
   static constexpr int oBar = oStg + kRows * D * 2;
   // barrier indices ([S buffer][half] for P, [half][buffer] for O)
   static constexpr int bQFull = 0, bQFree = bQFull + NQ, bKVFull = bQFree + NQ,
-                       bKVFree = bKVFull + NKV, bSFull = bKVFree + NKV, bSFree = bSFull + 2,
-                       bPFull = bSFree + 2, bPVDone = bPFull + 4, bOFull = bPVDone + 4,
+                       bKVFree = bKVFull + NKV, bSFull = bKVFree + NKV, bSFree = bSFull + NSB,
+                       bPFull = bSFree + NSB, bPVDone = bPFull + 2 * NSB, bOFull = bPVDone + 2 * NSB,
                        bOFree = bOFull + 2 * NOB, bXFull = bOFree + 2 * NOB, bXFree = bXFull + 2,
                        bDone = bXFree + 2, nBar = bDone + 1;
   static constexpr int oSlot = oBar + nBar * 8;
@@ -88,12 +91,15 @@ struct Cfg {
   static constexpr int kSmem = oSched + kSchedBytes + 1024;  // + slack for 1024-byte alignment
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   static constexpr uint32_t kTmemCols = 512;
-  // S buffers: columns [0,128) and [128,256).  Half h's P (64 keys, two bf16
+  // S buffer i: columns [128 i, 128 i + 128).  Half h's P (64 keys, two bf16
   // per column) overwrites the first 32 columns of that half's 64 S columns.
+  // The O accumulators follow (d = 64: 384 + 2 x 64 columns; d = 128: 256 +
+  // 2 x 128).
   static constexpr uint32_t tS = 0;
   __device__ static constexpr uint32_t tP(int sb, int h) { return tS + sb * kChunk + 64 * h; }
   // O accumulator of half h, buffer ob
-  __device__ static constexpr uint32_t tO(int h, int ob) { return 256 + (h * NOB + ob) * D; }
+  __device__ static constexpr uint32_t tO(int h, int ob) { return NSB * kChunk + (h * NOB + ob) * D; }
+  static_assert(NSB * kChunk + 2 * NOB * D <= kTmemCols, "tensor memory columns");
   // registers per thread after reallocation: TMA/MMA warpgroup, each softmax
   // warpgroup, epilogue warpgroup (the 16 warps share the 64K-register file)
   static constexpr int kRegsCtl = 56;
@@ -186,8 +192,8 @@ __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const 
   return 0;
 }
 
-// S = Q K^T for every chunk into S buffer G % 2 (warp 1, one thread).  P of
-// chunk G replaces S in that buffer, so S of chunk G + 2 waits for P V of
+// S = Q K^T for every chunk into S buffer G % NSB (warp 1, one thread).  P of
+// chunk G replaces S in that buffer, so S of chunk G + NSB waits for P V of
 // chunk G, which the other issuer signals on bSFree.
 template <int D>
 __device__ int s_issuer(const Params& p, const Sched& sch, uint32_t base, uint32_t tmem) {
@@ -202,11 +208,11 @@ __device__ int s_issuer(const Params& p, const Sched& sch, uint32_t base, uint32
     if (!mbar_wait(bar + 8 * (C::bQFull + qs), (tc / C::NQ) & 1)) return kErrQFull;
     const uint64_t dQ = smem_desc_sw128(base + C::oQ + qs * C::kQBytes, 0, 1024);
     for (int c = 0; c < x.nch; ++c) {
-      const int G = g + c, st = G % C::NKV, sb = G % 2;
+      const int G = g + c, st = G % C::NKV, sb = G % C::NSB;
       const uint64_t dK = smem_desc_sw128(base + C::oK + st * C::kKBytes, 0, 1024);
       const uint32_t tD = tmem + C::tS + sb * kChunk;
       if (!mbar_wait(bar + 8 * (C::bKVFull + st), (G / C::NKV) & 1)) return kErrKVFull;
-      if (!mbar_wait(bar + 8 * (C::bSFree + sb), ((G / 2) & 1) ^ 1)) return kErrSFree;
+      if (!mbar_wait(bar + 8 * (C::bSFree + sb), ((G / C::NSB) & 1) ^ 1)) return kErrSFree;
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
@@ -236,7 +242,7 @@ __device__ int pv_issuer(const Params& p, const Sched& sch, uint32_t base, uint3
     if (x.nch == 0) continue;
     const int ob = tc % C::NOB;
     for (int c = 0; c < x.nch; ++c) {
-      const int G = g + c, st = G % C::NKV, sb = G % 2;
+      const int G = g + c, st = G % C::NKV, sb = G % C::NSB;
       // V is MN-major: 64-column swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
       const uint64_t dV = smem_desc_sw128(base + C::oV + st * C::kKBytes, kSlab, 1024);
 #pragma unroll
@@ -245,7 +251,7 @@ __device__ int pv_issuer(const Params& p, const Sched& sch, uint32_t base, uint3
         if (c == 0 &&
             !mbar_wait(bar + 8 * (C::bOFree + h * C::NOB + ob), ((tc / C::NOB) & 1) ^ 1))
           return kErrOFree;
-        if (!mbar_wait(bar + 8 * (C::bPFull + 2 * sb + h), (G >> 1) & 1)) return kErrPFull;
+        if (!mbar_wait(bar + 8 * (C::bPFull + 2 * sb + h), (G / C::NSB) & 1)) return kErrPFull;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 4; ++k)  // 16 keys = 8 P columns = 2048 bytes of V per step
@@ -297,8 +303,8 @@ __device__ int softmax_warps(const Params& p, const Sched& sch, uint32_t base, u
     const int ob = tc % C::NOB;
     float m_used = -INFINITY, l = 0.f;
     for (int c = 0; c < x.nch; ++c) {
-      const int G = g + c, sb = G % 2;
-      if (!all_ok(mbar_wait(bar + 8 * (C::bSFull + sb), (G / 2) & 1))) return kErrSFull;
+      const int G = g + c, sb = G % C::NSB;
+      if (!all_ok(mbar_wait(bar + 8 * (C::bSFull + sb), (G / C::NSB) & 1))) return kErrSFull;
       tc_fence_after();
       float s[2][32];
 #pragma unroll
@@ -363,7 +369,7 @@ __device__ int softmax_warps(const Params& p, const Sched& sch, uint32_t base, u
         // this half's previous P V product must have landed before its O is rescaled
         // (need implies c > 0, so chunk G - 1 belongs to this tile)
         const int Gp = G - 1;
-        if (!all_ok(mbar_wait(bar + 8 * (C::bPVDone + 2 * (Gp % 2) + hf), (Gp >> 1) & 1)))
+        if (!all_ok(mbar_wait(bar + 8 * (C::bPVDone + 2 * (Gp % C::NSB) + hf), (Gp / C::NSB) & 1)))
           return kErrPPrev;
         tc_fence_after();
         const uint32_t to = trow + C::tO(hf, ob);
@@ -507,13 +513,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar + 8 * (C::bKVFull + i), 1);
       mbar_init(bar + 8 * (C::bKVFree + i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NSB; ++i) {
       mbar_init(bar + 8 * (C::bSFull + i), 1);
       mbar_init(bar + 8 * (C::bSFree + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(bar + 8 * (C::bXFull + i), 256);
       mbar_init(bar + 8 * (C::bXFree + i), 128);
     }
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2 * C::NSB; ++i) {
       mbar_init(bar + 8 * (C::bPFull + i), 128);
       mbar_init(bar + 8 * (C::bPVDone + i), 1);
     }

@@ -13,9 +13,12 @@
 // so the key/value blocks their windows share are served from L2.
 //
 // Warp roles (512 threads, four warpgroups with reallocated registers):
-//   warp 0     TMA producer: Q tile, then K and V chunks, into 128-byte
-//              swizzled shared memory (3-D tensor maps; rows outside [0, n)
-//              are zero-filled by TMA and masked).
+//   warp 0     TMA producer: Q tile, then K chunks, into 128-byte swizzled
+//              shared memory (3-D tensor maps; rows outside [0, n) are
+//              zero-filled by TMA and masked).  A K stage is freed as soon as
+//              its S product completes.
+//   warp 3     TMA producer of the V chunks (a V stage is freed by the P V
+//              products, later than the K stage of the same chunk).
 //   warp 1     TMEM owner and S issuer (one thread):
 //                S_c = Q K_c^T   (M 128, N 128, K d)   -> TMEM, three buffers at
 //                d = 64 (S of chunks c + 1 and c + 2 in flight while chunk c's
@@ -67,7 +70,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 template <int D>
 struct Cfg {
   static constexpr int NQ = D == 64 ? 2 : 1;   // Q tile buffers
-  static constexpr int NKV = D == 64 ? 3 : 2;  // K/V chunk stages
+  static constexpr int NKV = D == 64 ? 3 : 2;  // K chunk stages, and as many V chunk stages
   static constexpr int NSB = D == 64 ? 3 : 2;  // S buffers
   static constexpr int NOB = 1;  // O accumulators per half (tiles in flight)
   static constexpr int kQBytes = kRows * D * 2;
@@ -78,8 +81,9 @@ struct Cfg {
   static constexpr int oStg = oV + NKV * kKBytes;  // output tile staging (D / 64 boxes)
   static constexpr int oBar = oStg + kRows * D * 2;
   // barrier indices ([S buffer][half] for P, [half][buffer] for O)
-  static constexpr int bQFull = 0, bQFree = bQFull + NQ, bKVFull = bQFree + NQ,
-                       bKVFree = bKVFull + NKV, bSFull = bKVFree + NKV, bSFree = bSFull + NSB,
+  static constexpr int bQFull = 0, bQFree = bQFull + NQ, bKFull = bQFree + NQ,
+                       bKFree = bKFull + NKV, bVFull = bKFree + NKV, bVFree = bVFull + NKV,
+                       bSFull = bVFree + NKV, bSFree = bSFull + NSB,
                        bPFull = bSFree + NSB, bPVDone = bPFull + 2 * NSB, bOFull = bPVDone + 2 * NSB,
                        bOFree = bOFull + 2 * NOB, bXFull = bOFree + 2 * NOB, bXFree = bXFull + 2,
                        bDone = bXFree + 2, nBar = bDone + 1;
@@ -154,8 +158,8 @@ __device__ __forceinline__ Item sched_item(const Params& p, const Sched& s, int 
 }
 
 // error codes: 0x10 + site
-enum : int { kErrQFree = 0x11, kErrKVFree, kErrQFull, kErrKVFull, kErrSFree, kErrOFree, kErrPFull,
-             kErrSFull, kErrPPrev = 0x1a, kErrOFull, kErrDone, kErrXFull = 0x1e, kErrXFree };
+enum : int { kErrQFree = 0x11, kErrKFree, kErrQFull, kErrKFull, kErrSFree, kErrOFree, kErrPFull,
+             kErrSFull, kErrPPrev = 0x1a, kErrOFull, kErrDone, kErrXFull = 0x1e, kErrXFree, kErrVFree, kErrVFull };
 
 template <int D>
 __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tq,
@@ -176,18 +180,43 @@ __device__ int producer(const Params& p, const Sched& sch, uint32_t base, const 
                   s * 64, x.tile * kRows, bh);
     for (int c = 0; c < x.nch; ++c) {
       const int G = g + c, st = G % C::NKV;
-      if (!mbar_wait(bar + 8 * (C::bKVFree + st), ((G / C::NKV) & 1) ^ 1)) return kErrKVFree;
-      const uint32_t full = bar + 8 * (C::bKVFull + st);
-      mbar_arrive_expect_tx(full, 2 * C::kKBytes);
+      if (!mbar_wait(bar + 8 * (C::bKFree + st), ((G / C::NKV) & 1) ^ 1)) return kErrKFree;
+      const uint32_t full = bar + 8 * (C::bKFull + st);
+      mbar_arrive_expect_tx(full, C::kKBytes);
       const int y = (x.J0 + 4 * c) * kBlock;
 #pragma unroll
-      for (int s = 0; s < D / 64; ++s) {
+      for (int s = 0; s < D / 64; ++s)
         tma_load_3d(base + C::oK + st * C::kKBytes + s * kSlab, tk, full, s * 64, y, bh);
-        tma_load_3d(base + C::oV + st * C::kKBytes + s * kSlab, tv, full, s * 64, y, bh);
-      }
     }
     g += x.nch;
     ++tc;
+  }
+  return 0;
+}
+
+// V chunks (warp 3, one thread).  A V stage is freed by the chunk's P V
+// products, a K stage already by its S product, so the two streams run on
+// their own: the next K chunks load while earlier P V products still read V.
+template <int D>
+__device__ int v_producer(const Params& p, const Sched& sch, uint32_t base, const CUtensorMap* tv) {
+  using C = Cfg<D>;
+  const uint32_t bar = base + C::oBar;
+  int g = 0;
+  for (int it = blockIdx.x; it < sch.count; it += gridDim.x) {
+    const Item x = sched_item(p, sch, it);
+    if (x.nch == 0) continue;
+    const int bh = x.b * p.a.heads + x.h;
+    for (int c = 0; c < x.nch; ++c) {
+      const int G = g + c, st = G % C::NKV;
+      if (!mbar_wait(bar + 8 * (C::bVFree + st), ((G / C::NKV) & 1) ^ 1)) return kErrVFree;
+      const uint32_t full = bar + 8 * (C::bVFull + st);
+      mbar_arrive_expect_tx(full, C::kKBytes);
+      const int y = (x.J0 + 4 * c) * kBlock;
+#pragma unroll
+      for (int s = 0; s < D / 64; ++s)
+        tma_load_3d(base + C::oV + st * C::kKBytes + s * kSlab, tv, full, s * 64, y, bh);
+    }
+    g += x.nch;
   }
   return 0;
 }
@@ -211,7 +240,7 @@ __device__ int s_issuer(const Params& p, const Sched& sch, uint32_t base, uint32
       const int G = g + c, st = G % C::NKV, sb = G % C::NSB;
       const uint64_t dK = smem_desc_sw128(base + C::oK + st * C::kKBytes, 0, 1024);
       const uint32_t tD = tmem + C::tS + sb * kChunk;
-      if (!mbar_wait(bar + 8 * (C::bKVFull + st), (G / C::NKV) & 1)) return kErrKVFull;
+      if (!mbar_wait(bar + 8 * (C::bKFull + st), (G / C::NKV) & 1)) return kErrKFull;
       if (!mbar_wait(bar + 8 * (C::bSFree + sb), ((G / C::NSB) & 1) ^ 1)) return kErrSFree;
       tc_fence_after();
 #pragma unroll
@@ -220,6 +249,7 @@ __device__ int s_issuer(const Params& p, const Sched& sch, uint32_t base, uint32
         mma_bf16_ss(tD, desc_add(dQ, off), desc_add(dK, off), kIdS, k > 0);
       }
       mma_commit(bar + 8 * (C::bSFull + sb));
+      mma_commit(bar + 8 * (C::bKFree + st));  // the S product was this K chunk's only reader
       if (c == x.nch - 1) mma_commit(bar + 8 * (C::bQFree + qs));  // the tile's S products issued
     }
     g += x.nch;
@@ -245,6 +275,7 @@ __device__ int pv_issuer(const Params& p, const Sched& sch, uint32_t base, uint3
       const int G = g + c, st = G % C::NKV, sb = G % C::NSB;
       // V is MN-major: 64-column swizzle atoms kSlab apart, 8-key groups 1024 bytes apart
       const uint64_t dV = smem_desc_sw128(base + C::oV + st * C::kKBytes, kSlab, 1024);
+      if (!mbar_wait(bar + 8 * (C::bVFull + st), (G / C::NKV) & 1)) return kErrVFull;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {  // each half's 64 keys into its own O accumulator
         const uint32_t tO = tmem + C::tO(h, ob), tP = tmem + C::tP(sb, h);
@@ -260,7 +291,7 @@ __device__ int pv_issuer(const Params& p, const Sched& sch, uint32_t base, uint3
         if (c == x.nch - 1) mma_commit(bar + 8 * (C::bOFull + h * C::NOB + ob));
       }
       mma_commit(bar + 8 * (C::bSFree + sb));
-      mma_commit(bar + 8 * (C::bKVFree + st));
+      mma_commit(bar + 8 * (C::bVFree + st));
     }
     g += x.nch;
     ++tc;
@@ -510,8 +541,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar + 8 * (C::bQFree + i), 1);
     }
     for (int i = 0; i < C::NKV; ++i) {
-      mbar_init(bar + 8 * (C::bKVFull + i), 1);
-      mbar_init(bar + 8 * (C::bKVFree + i), 1);
+      mbar_init(bar + 8 * (C::bKFull + i), 1);
+      mbar_init(bar + 8 * (C::bKFree + i), 1);
+      mbar_init(bar + 8 * (C::bVFull + i), 1);
+      mbar_init(bar + 8 * (C::bVFree + i), 1);
     }
     for (int i = 0; i < C::NSB; ++i) {
       mbar_init(bar + 8 * (C::bSFull + i), 1);
@@ -558,6 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) err = producer<D>(p, sch, base, &tq, &tk, &tv);
     if (warp == 1 && lane == 0) err = s_issuer<D>(p, sch, base, tmem);
     if (warp == 2 && lane == 0) err = pv_issuer<D>(p, sch, base, tmem);
+    if (warp == 3 && lane == 0) err = v_producer<D>(p, sch, base, &tv);
   } else if (warp < 12) {
     regs_inc<C::kRegsSoft>();
     err = softmax_warps<D, kCausal>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);

@@ -230,7 +230,8 @@ def _full_size_windows(w, width, seed):
     plus windows on the persistent kernels' last wave of work items (one
     128-row tile per item, items handed round-robin to one CTA per SM): the
     wave's first tile, its middle and the sequence's last tile, where each
-    CTA runs its final item and its deferred epilogue."""
+    CTA runs its final item and the epilogue of that item (the forward's
+    epilogue warpgroup, the backward's deferred dK/dV epilogue)."""
     nb = w.n // BLOCK
     rng = np.random.default_rng(seed)
     out = []

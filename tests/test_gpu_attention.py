@@ -11,7 +11,8 @@ import numpy as np
 import pytest
 import torch
 
-from block_sparse_local_nb_b200.inputs import WORKLOADS, make_attn_inputs, random_attn_inputs
+from block_sparse_local_nb_b200.inputs import (WORKLOADS, AttnWorkload, make_attn_inputs,
+                                               random_attn_inputs)
 from oracle import attn_bwd_banded, attn_fwd_banded, attn_fwd_dense
 from tests.gpu_util import (ATOL_F32, GRAD_RFRO_BF16, LSE_ATOL_BF16, O_ATOL_BF16, f64, max_abs,
                             rel_fro, run_bwd, run_fwd, window)
@@ -218,6 +219,32 @@ def test_bf16_varlen_workload(name):
         edge = (Lb - 1) // BLOCK
         h = int(rng.integers(w.heads))
         _check_window(w, tensors, outs, (b, h), max(0, edge - 3), min(nb, edge + 4), lengths)
+    for t in outs:
+        for b in range(w.batch):
+            Lb = int(lengths[b])
+            assert (t[b, :, Lb:] == 0).all() or torch.isneginf(t[b, :, Lb:]).all()
+
+
+def test_bf16_d128_ragged_many_items():
+    """bf16, 6 x 8 x 8192 x 128, R = 3, lengths ~ U[1500, 8192]: about 21 work
+    items per CTA with empty tiles, so every role of both d = 128 kernels wraps
+    its buffer and barrier parities many times over ragged items.  Two whole
+    heads, each sequence's length boundary and the last wave of items."""
+    w = AttnWorkload("bf16_d128_ragged", "bf16", 6, 8, 8192, 128, 3, 5, varlen=(1500, 8192),
+                     desc="fwd+bwd bf16 6x8x8192x128 R=3 L~U[1500,8192]")
+    tensors, outs, lengths = _run_workload(w)
+    nb = w.n // BLOCK
+    for bh in [(0, 3), (5, 7)]:
+        _check_window(w, tensors, outs, bh, 0, nb, lengths)
+    rng = np.random.default_rng(3)
+    for b in range(w.batch):
+        edge = (int(lengths[b]) - 1) // BLOCK
+        _check_window(w, tensors, outs, (b, int(rng.integers(w.heads))), max(0, edge - 3),
+                      min(nb, edge + 4), lengths)
+    # the last non-empty tile of the last sequence, every head
+    edge = (int(lengths[-1]) - 1) // BLOCK
+    for h in range(w.heads):
+        _check_window(w, tensors, outs, (w.batch - 1, h), max(0, edge - 7), edge + 1, lengths)
     for t in outs:
         for b in range(w.batch):
             Lb = int(lengths[b])

@@ -43,6 +43,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 512;
+constexpr int kLaunchRegs = 65536 / kThreads / 8 * 8;  // per thread at launch
 
 constexpr int kRows = 128;        // keys per item, queries per chunk
 constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 128 bytes
@@ -601,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Role branches never join again: each ends with the CTA barrier, after which
   // warp 1 waits for the tensor cores and frees the TMEM.
   if (warp < 4) {
-    regs_dec<C::kRegsCtl>();
+    regs_dec<C::kRegsCtl, kLaunchRegs>();
     int err = 0;
     if (warp == 0 && lane == 0) err = producer<D>(p, sch, base, &tk, &tv, &tq, &tdo);
     if (warp == 1 && lane == 0) err = sdp_issuer<D>(p, sch, base, tmem);
@@ -621,14 +622,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_dealloc(tmem, C::kTmemCols);
     }
   } else if (warp < 12) {
-    regs_inc<C::kRegsGrad>();
+    regs_inc<C::kRegsGrad, kLaunchRegs>();
     const int err =
         grad_warps<D, kCausal>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
     if (err) record_error(p.a.err, err);
     pdl_trigger();  // this CTA's work is issued: the next kernel may start launching
     __syncthreads();
   } else {
-    regs_dec<C::kRegsDq>();
+    regs_dec<C::kRegsDq, kLaunchRegs>();
     const int err = dq_warps<D>(p, sch, base, gbase, tmem, warp & 3, lane, &tdq);
     if (err) record_error(p.a.err, err);
     pdl_trigger();  // this CTA's work is issued: the next kernel may start launching

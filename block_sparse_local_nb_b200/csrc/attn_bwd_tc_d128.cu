@@ -44,6 +44,7 @@ using namespace sm100;
 
 constexpr int D = 128;
 constexpr int kThreads = 512;
+constexpr int kLaunchRegs = 65536 / kThreads / 8 * 8;  // per thread at launch
 constexpr int kKeys = 128;  // keys per item
 constexpr int kQ = 64;      // queries per chunk (two query blocks)
 constexpr int kNS = 3;      // Q/dO stages
@@ -516,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Role branches never join again: each ends with the CTA barrier, after which
   // warp 1 waits for the tensor cores and frees the TMEM.
   if (warp < 4) {
-    regs_dec<kRegsCtl>();
+    regs_dec<kRegsCtl, kLaunchRegs>();
     int err = 0;
     if (warp == 0 && lane == 0) err = producer(p, sch, base, &tk, &tv, &tq, &tdo);
     if (warp == 1 && lane == 0) err = sdp_issuer(p, sch, base, tmem);
@@ -536,13 +537,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_dealloc(tmem, kTmemCols);
     }
   } else if (warp < 12) {
-    regs_inc<kRegsGrad>();
+    regs_inc<kRegsGrad, kLaunchRegs>();
     const int err = grad_warps<kCausal>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
     if (err) record_error(p.a.err, err);
     pdl_trigger();
     __syncthreads();
   } else {
-    regs_dec<kRegsDq>();
+    regs_dec<kRegsDq, kLaunchRegs>();
     const int err = dq_warps(p, sch, base, gbase, tmem, warp & 3, lane, &tdq);
     if (err) record_error(p.a.err, err);
     pdl_trigger();

@@ -60,6 +60,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 512;
+constexpr int kLaunchRegs = 65536 / kThreads / 8 * 8;  // per thread at launch
 constexpr int kRows = 128;   // query rows per tile
 constexpr int kChunk = 128;  // keys per chunk
 constexpr int kSlab = 128 * 128;  // one swizzled box: 128 rows x 64 bf16
@@ -588,16 +589,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   int err = 0;
   if (warp < 4) {
-    regs_dec<C::kRegsCtl>();
+    regs_dec<C::kRegsCtl, kLaunchRegs>();
     if (warp == 0 && lane == 0) err = producer<D>(p, sch, base, &tq, &tk, &tv);
     if (warp == 1 && lane == 0) err = s_issuer<D>(p, sch, base, tmem);
     if (warp == 2 && lane == 0) err = pv_issuer<D>(p, sch, base, tmem);
     if (warp == 3 && lane == 0) err = v_producer<D>(p, sch, base, &tv);
   } else if (warp < 12) {
-    regs_inc<C::kRegsSoft>();
+    regs_inc<C::kRegsSoft, kLaunchRegs>();
     err = softmax_warps<D, kCausal>(p, sch, base, gbase, tmem, warp & 3, (warp - 4) >> 2, lane);
   } else {
-    regs_dec<C::kRegsEpi>();
+    regs_dec<C::kRegsEpi, kLaunchRegs>();
     err = epi_warps<D>(p, sch, base, gbase, tmem, warp & 3, lane, &to);
   }
   if (err) record_error(p.a.err, err);

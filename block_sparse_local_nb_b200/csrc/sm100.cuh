@@ -241,13 +241,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 
-// Per-warpgroup register reallocation (all four warps of a warpgroup execute it).
-template <int N>
+// Per-warpgroup register reallocation (all four warps of a warpgroup execute
+// it).  L is the per-thread count the kernel was launched with: a decrease may
+// not go above it, an increase not below it.
+template <int N, int L>
 __device__ __forceinline__ void regs_dec() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= L, "setmaxnreg.dec count");
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
-template <int N>
+template <int N, int L>
 __device__ __forceinline__ void regs_inc() {
+  static_assert(N % 8 == 0 && N <= 256 && N >= L, "setmaxnreg.inc count");
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
